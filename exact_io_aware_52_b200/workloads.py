@@ -1,0 +1,103 @@
+"""Seeded synthetic inputs for the attention forward pass.
+
+This module only draws random numbers and describes problem shapes; it holds
+none of the attention arithmetic.  It is the one module that both the CUDA
+path's callers (tests, bench) and the fp64 oracle's callers share.
+
+Recipe (every workload): a CPU ``torch.Generator`` seeded with ``seed``; Q, K
+and V drawn in that order as float32 ``randn`` of shape [B, H, N, d] times the
+stated standard deviation, then rounded to bfloat16 (round-to-nearest-even);
+for key-padded workloads the per-sequence key lengths are drawn next as
+integers uniform in [lo, hi] inclusive.  The scale is the float32 value of
+1/sqrt(d).  The shapes stand in for the pages' BERT-large (length 512) and
+GPT-2 (length 1K) workloads by shape only; no dataset is involved.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    qk_std: float = 1.0
+    kpad: tuple | None = None          # (lo, hi) inclusive range of key lengths, or None
+    sample_rows_per_head: int | None = None  # rows the oracle checks per head (None: all)
+    seed: int = 0
+    notes: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        # the float32 value the kernel receives, as a Python float
+        return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32).item())
+
+    def flops(self) -> float:
+        """Nominal attention FLOPs: 4*B*H*N^2*d, halved when causal."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+
+# The five workloads; seeds are 52000 + workload number.
+WORKLOADS = {
+    1: Workload("tiny B1 H1 N128 d64 non-causal", 1, 1, 128, 64, False, seed=52001),
+    2: Workload("gpt2-small-shaped B8 H12 N1024 d64 causal", 8, 12, 1024, 64, True, seed=52002),
+    3: Workload("bert-large-shaped B16 H16 N512 d64 key-padded L~U[256,512]", 16, 16, 512, 64,
+                False, kpad=(256, 512), seed=52003),
+    4: Workload("long-context causal B1 H32 N16384 d128", 1, 32, 16384, 128, True,
+                sample_rows_per_head=512, seed=52004),
+    5: Workload("softmax-stress causal B1 H16 N65536 d128 QK~N(0,4^2)", 1, 16, 65536, 128, True,
+                qk_std=4.0, sample_rows_per_head=256, seed=52005),
+}
+
+
+def make_inputs(w: Workload, seed: int | None = None):
+    """Draw (q, k, v, k_len) on the CPU for workload ``w``.
+
+    q, k, v: bfloat16 [B, H, N, d] contiguous CPU tensors.
+    k_len: int32 [B] CPU tensor, or None when the workload has no key padding.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    shape = (w.B, w.H, w.N, w.d)
+    q = (torch.randn(shape, generator=g, dtype=torch.float32) * w.qk_std).to(torch.bfloat16)
+    k = (torch.randn(shape, generator=g, dtype=torch.float32) * w.qk_std).to(torch.bfloat16)
+    v = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k_len = None
+    if w.kpad is not None:
+        lo, hi = w.kpad
+        k_len = torch.randint(lo, hi + 1, (w.B,), generator=g, dtype=torch.int64).to(torch.int32)
+    return q, k, v, k_len
+
+
+def sample_rows(w: Workload, seed: int | None = None):
+    """Flat row ids (b*H + h)*N + i the oracle checks for ``w``.
+
+    All rows when ``w.sample_rows_per_head`` is None; otherwise, per (b, h), a
+    seeded uniform sample without replacement of that many query rows, plus
+    rows 0 and N-1, sorted.
+    """
+    import numpy as np
+
+    n_bh = w.B * w.H
+    if w.sample_rows_per_head is None:
+        return np.arange(n_bh * w.N, dtype=np.int64)
+    rng = np.random.default_rng((w.seed if seed is None else seed) + 7)
+    out = []
+    for bh in range(n_bh):
+        pick = rng.choice(w.N, size=min(w.sample_rows_per_head, w.N), replace=False)
+        pick = np.union1d(pick, [0, w.N - 1])
+        out.append(bh * w.N + pick.astype(np.int64))
+    return np.concatenate(out)
+
+
+def custom(B, H, N, d, causal, qk_std=1.0, kpad=None, seed=1, name="custom") -> Workload:
+    """A workload of arbitrary shape (tests of ragged and edge shapes)."""
+    return Workload(name, B, H, N, d, causal, qk_std=qk_std, kpad=kpad, seed=seed)

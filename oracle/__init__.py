@@ -1,0 +1,122 @@
+"""fp64 CPU oracle for the exact attention forward pass.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are the only callers.  The CUDA product path
+never imports this package, and this package imports nothing from it.
+
+Two pieces, both written from the page "FlashAttention (ES)":
+
+* ``attention_f64`` -- the plain definition of attention (section "El problema
+  de la atencion estandar", the Attention equation, with the masking step of
+  section "Fusion de operaciones en un unico kernel de CUDA"), computed in C
+  with OpenMP over rows in ``attn_oracle.c``: full score row, mask,
+  max-subtracted softmax, weighted sum of V rows.
+* ``online.attention_online`` -- the tiled online-softmax recurrence of
+  section "Calculo de Softmax en linea" in pure Python, used only on tiny
+  inputs to pin the recurrence against the two-pass definition.
+
+Pinned by ``tests/test_oracle.py`` against closed forms, invariants, a
+library routine (torch's fp64 scaled-dot-product attention) and brute force.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile the C oracle (``attn_oracle.c`` by default) into a shared library.
+
+    No fast-math: the oracle keeps IEEE double semantics.
+    """
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-Wall", "-Wextra",
+             "-fno-fast-math", src, "-o", tmp, "-lm"])
+        os.replace(tmp, out)
+    return out
+
+
+def load_library(path: str):
+    """ctypes handle on a built oracle library with its signature declared."""
+    lib = ctypes.CDLL(path)
+    f = lib.attn_oracle_f64
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
+                  ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = load_library(build())
+    return _lib
+
+
+def _as_bf16_bits(x) -> np.ndarray:
+    """Accept a torch bf16 tensor (CPU) or a numpy uint16 array of bf16 bits."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint16:
+            raise TypeError("numpy inputs must be uint16 bf16 bit patterns")
+        return np.ascontiguousarray(x)
+    import torch  # only for the bit view of a bf16 tensor
+    if x.dtype != torch.bfloat16:
+        raise TypeError("torch inputs must be bfloat16")
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def attention_f64(q, k, v, causal: bool, scale: float, k_len=None, rows=None,
+                  nthreads: int | None = None, lib=None):
+    """Exact attention in fp64 from bf16 inputs.
+
+    q, k, v: [B, H, N, d] bf16 (torch CPU tensor or uint16 bit array).
+    causal: key j is masked for query i when j > i.
+    scale: the float32 multiplier of q.k (the definition's 1/sqrt(d_k)).
+    k_len: None or int sequence of length B; key j of batch b masked iff j >= k_len[b].
+    rows: None (all rows) or int64 flat row ids (b*H + h)*N + i.
+    lib: a library from ``load_library`` (default: the built ``attn_oracle.c``).
+    Returns (O [n_rows, d] float64, lse [n_rows] float64); n_rows = B*H*N when
+    rows is None (row r = (b*H + h)*N + i).
+    """
+    qb, kb, vb = _as_bf16_bits(q), _as_bf16_bits(k), _as_bf16_bits(v)
+    if qb.ndim != 4 or qb.shape != kb.shape or qb.shape != vb.shape:
+        raise ValueError("q, k, v must share one [B, H, N, d] shape")
+    B, H, N, d = qb.shape
+    kl = None
+    if k_len is not None:
+        kl = np.ascontiguousarray(np.asarray(k_len, dtype=np.int32).reshape(-1))
+        if kl.shape[0] != B:
+            raise ValueError("k_len must have B entries")
+    if rows is None:
+        n_rows = B * H * N
+        rr = None
+    else:
+        rr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        n_rows = rr.shape[0]
+    o = np.zeros((n_rows, d), dtype=np.float64)
+    lse = np.zeros((n_rows,), dtype=np.float64)
+    nt = nthreads if nthreads is not None else (os.cpu_count() or 1)
+    lib = _load() if lib is None else lib
+    rc = lib.attn_oracle_f64(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
+        None if kl is None else kl.ctypes.data, B, H, N, d, int(bool(causal)),
+        ctypes.c_float(scale), None if rr is None else rr.ctypes.data,
+        n_rows, o.ctypes.data, lse.ctypes.data, int(nt))
+    if rc != 0:
+        raise RuntimeError(f"attn_oracle_f64 failed with code {rc}")
+    return o, lse

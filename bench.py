@@ -1,0 +1,413 @@
+"""Benchmark of the fused sm_100a attention forward (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ours|reference]
+
+A step is one launch of the fused kernel over the whole workload: every
+(b, h, query tile) unit, i.e. every step of the hot path.  Inputs are
+resident in HBM when the timed region starts and are larger than L2 (the
+default workload reads 403 MB of Q, K, V; L2 is 126 MB), so no explicit
+flush is needed.  Timing: W untimed warm-up steps, then K steps bracketed by
+a barrier and a device synchronise on both sides, measured with CUDA events
+on the launching stream, max over ranks.
+
+Metric: attention forward TFLOP/s with FLOPs = 4*B*H*N^2*d (halved when
+causal), bf16 operands with fp32 accumulation, whole job over all ranks.
+With N GPUs each rank runs its own replica of the workload (the units are
+independent; no collective on the data path): weak scaling.
+
+`--impl reference` times the fp64 CPU oracle instead (the method's plain
+definition on the host cores), each step a bounded sample of query rows of
+the same workload, reported in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_52_b200 import _binding as fb  # noqa: E402
+from exact_io_aware_52_b200 import workloads  # noqa: E402
+
+DEFAULT_WORKLOAD = 4  # long-context causal B1 H32 N16384 d128: the tensor-bound headline
+METRIC = "attention fwd TFLOP/s (bf16, 1xB200) and % of dense BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["fa_fwd_kernel.cuh", "sm100_ptx.cuh", "fa_api.cu"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "exact_io_aware_52_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload_id: int):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "fa_fwd_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    rec = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            k, _, v = line.partition(" ")
+            rec[k] = v.strip()
+    if rec.get("source_hash") != kernel_source_hash() or rec.get("workload") != str(workload_id):
+        return None
+    try:
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def algorithmic_bytes(w, k_len) -> float:
+    """Compulsory HBM bytes of one launch: Q, K, V read once (valid keys only
+    under key padding), O (fp32) and lse written once."""
+    n_elem = w.B * w.H * w.N * w.d
+    kv_rows = w.H * (sum(min(max(int(x), 0), w.N) for x in k_len) if k_len is not None else w.B * w.N)
+    return 2.0 * n_elem + 2 * 2.0 * kv_rows * w.d + 4.0 * n_elem + 4.0 * w.B * w.H * w.N
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        props = torch.cuda.get_device_properties(device_index)
+        self.bus = None
+        try:
+            self.bus = "%08X:%02X:%02X" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+        except AttributeError:
+            pass
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) != len(self.FIELDS):
+                    continue
+                if self.bus and not parts[0].upper().endswith(self.bus[-7:]):
+                    continue
+                rows.append(parts)
+        if not rows:
+            return None
+        try:
+            sm = [float(r[1]) for r in rows]
+            smax = max(float(r[2]) for r in rows)
+            power = [float(r[3]) for r in rows]
+        except ValueError:
+            return None
+        loaded = [r for r, p in zip(rows, power) if p > 0.5 * max(power)] or rows
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in loaded:
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(float(r[1]) for r in loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(power), "sm_mhz_min": min(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl != "ours":
+        return world, rank, local  # the reference arm runs on rank 0 alone, no process group
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_rows_flops(w, rows, k_len) -> float:
+    """Nominal FLOPs of the given rows: 4*d per allowed score."""
+    tot = 0
+    for r in rows:
+        bh, i = divmod(int(r), w.N)
+        b = bh // w.H
+        e = w.N if k_len is None else max(0, min(w.N, int(k_len[b])))
+        if w.causal:
+            e = min(e, i + 1)
+        tot += e
+    return 4.0 * w.d * tot
+
+
+def cpu_oracle_rate(w, q, k, v, k_len, budget_s: float, seed: int = 0):
+    """Time the fp64 oracle on rows of the workload for about budget_s seconds;
+    returns (TFLOP/s in the metric's unit, threads, description, seconds)."""
+    import numpy as np
+
+    import oracle
+    threads = os.cpu_count() or 1
+    rng = np.random.default_rng(seed)
+    n_rows = w.B * w.H * w.N
+    kl = None if k_len is None else k_len.tolist()
+    batch = max(threads, 8)
+    flops = 0.0
+    done = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        rows = np.sort(rng.choice(n_rows, size=min(batch, n_rows), replace=False)).astype(np.int64)
+        oracle.attention_f64(q, k, v, w.causal, w.scale, k_len=kl, rows=rows, nthreads=threads)
+        flops += oracle_rows_flops(w, rows, kl)
+        done += len(rows)
+    dt = time.perf_counter() - t0
+    desc = f"{done} uniformly sampled query rows of the workload (all keys of each row), {dt:.1f} s"
+    return flops / dt / 1e12, threads, desc, dt
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle, bounded sample per step."""
+    w = workloads.WORKLOADS[args.workload]
+    if rank != 0:
+        return  # rank 0 alone times the oracle
+    q, k, v, k_len = workloads.make_inputs(w)
+    import numpy as np
+
+    import oracle
+    threads = os.cpu_count() or 1
+    rng = np.random.default_rng(1)
+    kl = None if k_len is None else k_len.tolist()
+    rows_per_step = max(threads, 8)
+    n_rows = w.B * w.H * w.N
+
+    def step():
+        rows = np.sort(rng.choice(n_rows, size=rows_per_step, replace=False)).astype(np.int64)
+        oracle.attention_f64(q, k, v, w.causal, w.scale, k_len=kl, rows=rows, nthreads=threads)
+        return oracle_rows_flops(w, rows, kl)
+
+    for _ in range(args.warmup):
+        step()
+    flops = 0.0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        flops += step()
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "step": f"fp64 CPU oracle on {rows_per_step} sampled query rows"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows_per_step} uniformly sampled query rows per step, "
+                                   f"{args.steps} steps"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CUDA library has no CPU path)")
+    fb.load()
+    w = workloads.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    q, k, v, k_len = workloads.make_inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    kld = None if k_len is None else k_len.to(dev)
+    o = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.float32, device=dev)
+    lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    params = fb.make_params(qd, kd, vd, o, lse, w.causal, w.scale, k_len=kld)
+    lib = fb.load()
+    sptr = fb._stream(stream)
+    import ctypes
+    pref = ctypes.byref(params)
+
+    def launch():
+        st = lib.fa_fwd_ex(pref, sptr)
+        if st != fb.FA_OK:
+            raise fb.FaError(st, "fa_fwd_ex")
+
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            launch()
+    stream.synchronize()
+
+    # per-launch events on the launching stream (for the kernel's own duration)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            launch()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per_launch = [a.elapsed_time(b) for a, b in ev]
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    kernel_ms = max_over_ranks(statistics.mean(per_launch), world)
+
+    flops = w.flops()
+    total_flops = flops * args.steps * world
+    value = total_flops / (elapsed_ms * 1e-3) / 1e12
+
+    # end to end through the public C ABI on host buffers (copies included)
+    e2e = None
+    if args.e2e_steps > 0:
+        qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+        klh = None if k_len is None else k_len.pin_memory()
+        oh = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.float32).pin_memory()
+        lh = torch.empty(w.B, w.H, w.N, dtype=torch.float32).pin_memory()
+        fb.fa_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, w.causal, w.scale, k_len_h=klh, k_len_d=kld,
+                       stream=stream)
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            fb.fa_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, w.causal, w.scale, k_len_h=klh,
+                           k_len_d=kld, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        h2d = 3 * qh.numel() * 2 + (0 if klh is None else klh.numel() * 4)
+        d2h = oh.numel() * 4 + lh.numel() * 4
+        e2e = {"value": flops * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "ms_per_step": e2e_ms / args.e2e_steps}
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    alg_bytes = algorithmic_bytes(w, k_len)
+    traffic = measured_traffic(args.workload)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "kernel": "fa_fwd_sm100_kernel", "kernel_ms": kernel_ms,
+                "algorithmic_bytes": alg_bytes, "hbm_gbs_algorithmic": alg_bytes / (kernel_ms * 1e-3) / 1e9,
+                "hbm_peak_gbs": float(peaks["hbm_gbs"])}
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        rate, threads, desc, _ = cpu_oracle_rate(w, q, k, v, k_len, budget_s=15.0)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "out": "fp32 O + fp32 lse", "flops_per_step_per_gpu": flops,
+                   "l2": "inputs larger than L2 (Q,K,V %.0f MB > 126 MB); no flush" % (3 * q.numel() * 2 / 1e6),
+                   "parallelism": f"replicas x{world}"},
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,10 +1,13 @@
 """B200-native exact attention forward (FlashAttention-style) behind a C ABI.
 
-The hot path lives in ``csrc/`` (hand-written sm_100a CUDA, built into
-``libfa_sm100.so``); this package is a thin ctypes binding over that library
-plus the seeded workload generator.  Nothing here computes attention on the
-CPU: when the library is missing, calls fail loudly.
+The hot path lives in ``csrc/`` (hand-written sm_100a CUDA built into
+``libfa_sm100.so``, C ABI in ``include/fa.h``); this package is a thin ctypes
+binding over that library plus the seeded workload generator.  Nothing here
+computes attention on the CPU: when the library is missing, calls fail loudly.
 """
+from ._binding import (  # noqa: F401
+    FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT, FA_ERR_INVALID_ARGUMENT, FA_ERR_MISALIGNED, FA_ERR_UNSUPPORTED,
+    FA_FLAG_EAGER_RESCALE, FA_O_BF16, FA_O_F32, FA_OK, FaError, attention, fa_fwd, fa_fwd_ex, fa_fwd_host,
+    read_device_status, status_string, version,
+)
 from .workloads import WORKLOADS, Workload, make_inputs, sample_rows  # noqa: F401
-
-__all__ = ["WORKLOADS", "Workload", "make_inputs", "sample_rows"]

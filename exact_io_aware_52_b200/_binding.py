@@ -1,0 +1,185 @@
+"""ctypes binding over the C ABI of include/fa.h (libfa_sm100.so).
+
+Argument marshalling only: tensors are passed as raw device pointers and the
+current CUDA stream; every step of the computation runs in the CUDA library.
+torch supplies device memory and streams.  If the library is missing, every
+call raises -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa_sm100.so")
+SELFTEST_LIB_PATH = os.path.join(HERE, "libfa_selftest.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARGUMENT = 1
+FA_ERR_MISALIGNED = 2
+FA_ERR_UNSUPPORTED = 3
+FA_ERR_CUDA = 4
+FA_ERR_DEVICE_TIMEOUT = 5
+FA_O_F32 = 0
+FA_O_BF16 = 1
+FA_FLAG_EAGER_RESCALE = 1
+
+_lock = threading.Lock()
+_lib = None
+_selftest = None
+
+
+class FaParams(ctypes.Structure):
+    """Mirror of fa_fwd_params."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("k_len", ctypes.c_void_p),
+        ("dev_status", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int),
+        ("causal", ctypes.c_int), ("scale", ctypes.c_float), ("o_dtype", ctypes.c_int),
+        ("flags", ctypes.c_int), ("timeout_ms", ctypes.c_uint32),
+    ]
+
+
+class FaHostParams(ctypes.Structure):
+    """Mirror of fa_fwd_host_params."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("k_len", ctypes.c_void_p), ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("dev", FaParams),
+    ]
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed: {status_string(status)} ({status})")
+
+
+def load():
+    """Load libfa_sm100.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                                   "(run `python -m exact_io_aware_52_b200.build`)")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+            lib.fa_fwd.restype = i
+            lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+            lib.fa_fwd_ex.restype = i
+            lib.fa_fwd_ex.argtypes = [ctypes.POINTER(FaParams), vp]
+            lib.fa_fwd_host.restype = i
+            lib.fa_fwd_host.argtypes = [ctypes.POINTER(FaHostParams), vp]
+            lib.fa_read_device_status.restype = i
+            lib.fa_read_device_status.argtypes = [vp, vp]
+            lib.fa_status_string.restype = ctypes.c_char_p
+            lib.fa_status_string.argtypes = [i]
+            lib.fa_version.restype = i
+            lib.fa_version.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def load_selftest():
+    """Load libfa_selftest.so (raises if it has not been built)."""
+    global _selftest
+    with _lock:
+        if _selftest is None:
+            if not os.path.exists(SELFTEST_LIB_PATH):
+                raise RuntimeError(f"self-test library not built: {SELFTEST_LIB_PATH} is missing")
+            lib = ctypes.CDLL(SELFTEST_LIB_PATH)
+            vp, i = ctypes.c_void_p, ctypes.c_int
+            lib.fa_selftest_tma_sw128.restype = i
+            lib.fa_selftest_tma_sw128.argtypes = [vp, vp, vp, vp]
+            lib.fa_selftest_mma_ss.restype = i
+            lib.fa_selftest_mma_ss.argtypes = [vp, vp, vp, i, vp, vp]
+            lib.fa_selftest_mma_ts.restype = i
+            lib.fa_selftest_mma_ts.argtypes = [vp, vp, vp, i, vp, vp]
+            lib.fa_selftest_wait_timeout.restype = i
+            lib.fa_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
+            _selftest = lib
+    return _selftest
+
+
+def status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return load().fa_version()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(st: int, where: str):
+    if st != FA_OK:
+        raise FaError(st, where)
+
+
+def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
+    """fa_fwd: q, k, v bf16 [B,H,N,d] CUDA tensors; o fp32 [B,H,N,d]; lse fp32 [B,H,N]."""
+    B, H, N, d = q.shape
+    st = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, int(bool(causal)),
+                       ctypes.c_float(scale), _stream(stream))
+    _check(st, "fa_fwd")
+
+
+def make_params(q, k, v, o, lse, causal, scale, k_len=None, dev_status=None, flags=0, timeout_ms=0,
+                shape=None) -> FaParams:
+    """Fill a fa_fwd_params from tensors (any of them may be None for argument tests)."""
+    import torch
+    if shape is None:
+        shape = tuple(q.shape)
+    B, H, N, d = shape
+    o_dtype = FA_O_BF16 if (o is not None and o.dtype == torch.bfloat16) else FA_O_F32
+    return FaParams(q=_ptr(q), k=_ptr(k), v=_ptr(v), o=_ptr(o), lse=_ptr(lse), k_len=_ptr(k_len),
+                    dev_status=_ptr(dev_status), B=B, H=H, N=N, d=d, causal=int(bool(causal)),
+                    scale=float(scale), o_dtype=o_dtype, flags=int(flags), timeout_ms=int(timeout_ms))
+
+
+def fa_fwd_ex(q, k, v, o, lse, causal: bool, scale: float, k_len=None, dev_status=None, flags: int = 0,
+              timeout_ms: int = 0, stream=None):
+    """fa_fwd_ex: as fa_fwd, plus k_len (int32 [B] CUDA tensor), o may be bf16,
+    an optional int32 status word, FA_FLAG_* flags and the wait time limit."""
+    p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms)
+    _check(load().fa_fwd_ex(ctypes.byref(p), _stream(stream)), "fa_fwd_ex")
+
+
+def fa_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal: bool, scale: float,
+                k_len_h=None, k_len_d=None, dev_status=None, flags: int = 0, stream=None):
+    """fa_fwd_host: host (pinned) tensors in and out, device tensors as staging."""
+    dev = make_params(q_d, k_d, v_d, o_d, lse_d, causal, scale, k_len_d, dev_status, flags)
+    hp = FaHostParams(q=_ptr(q_h), k=_ptr(k_h), v=_ptr(v_h), k_len=_ptr(k_len_h), o=_ptr(o_h), lse=_ptr(lse_h),
+                      dev=dev)
+    _check(load().fa_fwd_host(ctypes.byref(hp), _stream(stream)), "fa_fwd_host")
+
+
+def read_device_status(dev_status, stream=None) -> int:
+    return load().fa_read_device_status(_ptr(dev_status), _stream(stream))
+
+
+def attention(q, k, v, causal: bool, scale: float, k_len=None, out_dtype=None, flags: int = 0, stream=None):
+    """Allocate O and lse with torch on q's device and run fa_fwd_ex.
+
+    Returns (O [B,H,N,d] in out_dtype (fp32 default), lse [B,H,N] fp32).
+    """
+    import torch
+    B, H, N, d = q.shape
+    o = torch.empty((B, H, N, d), dtype=out_dtype or torch.float32, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fa_fwd_ex(q, k, v, o, lse, causal, scale, k_len=k_len, flags=flags, stream=stream)
+    return o, lse

@@ -1,0 +1,236 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument validation, the
+// per-device property cache, TMA tensor-map encoding and the kernel launch.
+// The library allocates nothing: every buffer belongs to the caller.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_fwd_kernel.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool probed = false;
+    bool supported = false;
+    int num_sms = 0;
+    bool attr_set[2][2] = {{false, false}, {false, false}};  // [d==128][bf16 out]
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status load_encoder() {
+    if (g_encode) return FA_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return FA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return FA_OK;
+}
+
+// Device checks are cached per device ordinal.
+fa_status probe_device(int *dev_out, DeviceInfo **info_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    DeviceInfo &di = g_dev[dev];
+    if (!di.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FA_ERR_CUDA;
+        di.supported = (major == 10 && minor == 0);  // the binary is sm_100a only
+        di.num_sms = sms;
+        di.probed = true;
+    }
+    if (!di.supported) return FA_ERR_UNSUPPORTED;
+    *dev_out = dev;
+    *info_out = &di;
+    return FA_OK;
+}
+
+// 3-D map over a contiguous [B*H][N][D] bf16 tensor: dims innermost first
+// {D, N, B*H}; box {64, 128, 1} (one 128-byte column block of a 128-row
+// tile); 128-byte swizzle, the layout the tcgen05 descriptors describe.
+// Out-of-range rows read as zero.
+fa_status encode_map(CUtensorMap *map, const void *base, int BH, int N, int D) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)fa::BM, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Validation that needs no device: shared by every entry point.
+fa_status validate(const fa_fwd_params *p) {
+    if (!p) return FA_ERR_INVALID_ARGUMENT;
+    if (p->B < 0 || p->H < 0 || p->N < 0) return FA_ERR_INVALID_ARGUMENT;
+    if (!(std::isfinite(p->scale) && p->scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
+    if (p->causal != 0 && p->causal != 1) return FA_ERR_INVALID_ARGUMENT;
+    if (p->o_dtype != FA_O_F32 && p->o_dtype != FA_O_BF16) return FA_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~FA_FLAG_EAGER_RESCALE) return FA_ERR_INVALID_ARGUMENT;
+    if (p->d != 64 && p->d != 128) return FA_ERR_UNSUPPORTED;
+    const long long rows = (long long)p->B * p->H * p->N;
+    if (rows == 0) return FA_OK;
+    if ((long long)p->B * p->H > 0x7fffffffLL || (long long)p->B * p->H * ((p->N + 127) / 128) > 0x7fffffffLL)
+        return FA_ERR_INVALID_ARGUMENT;
+    if (!p->q || !p->k || !p->v || !p->o || !p->lse) return FA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v) || !aligned16(p->o)) return FA_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(p->lse) & 3u) || (reinterpret_cast<uintptr_t>(p->k_len) & 3u) ||
+        (reinterpret_cast<uintptr_t>(p->dev_status) & 3u))
+        return FA_ERR_MISALIGNED;
+    return FA_OK;
+}
+
+template <int D, bool BF16>
+fa_status launch(const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t stream) {
+    auto kern = fa::fa_fwd_sm100_kernel<D, BF16>;
+    const int smem = fa::Cfg<D>::kSmemBytes;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        bool &set = di.attr_set[D == 128][BF16];
+        if (!set) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+                return FA_ERR_CUDA;
+            set = true;
+        }
+    }
+    kern<<<grid, fa::kThreads, smem, stream>>>(kp);
+    return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
+    fa_status st = validate(p);
+    if (st != FA_OK) return st;
+    if ((long long)p->B * p->H * p->N == 0) return FA_OK;
+
+    int dev = 0;
+    DeviceInfo *di = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        st = probe_device(&dev, &di);
+        if (st == FA_OK) st = load_encoder();
+    }
+    if (st != FA_OK) return st;
+
+    fa::FwdParams kp;
+    std::memset(&kp, 0, sizeof kp);
+    const int BH = p->B * p->H;
+    if ((st = encode_map(&kp.tm_q, p->q, BH, p->N, p->d)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_k, p->k, BH, p->N, p->d)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_v, p->v, BH, p->N, p->d)) != FA_OK) return st;
+    kp.o = p->o;
+    kp.lse = p->lse;
+    kp.k_len = p->k_len;
+    kp.status = p->dev_status;
+    kp.B = p->B;
+    kp.H = p->H;
+    kp.N = p->N;
+    kp.n_qtiles = (p->N + fa::BM - 1) / fa::BM;
+    kp.n_tiles = BH * kp.n_qtiles;
+    kp.causal = p->causal;
+    kp.scale_log2 = (float)((double)p->scale * 1.4426950408889634074);
+    kp.tau = (p->flags & FA_FLAG_EAGER_RESCALE) ? 0.f : 8.f;
+    kp.timeout_ns = (uint64_t)(p->timeout_ms ? p->timeout_ms : 2000u) * 1000000ull;
+
+    const int grid = kp.n_tiles < di->num_sms ? kp.n_tiles : di->num_sms;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf16 = p->o_dtype == FA_O_BF16;
+    if (p->d == 64) return bf16 ? launch<64, true>(kp, *di, grid, s) : launch<64, false>(kp, *di, grid, s);
+    return bf16 ? launch<128, true>(kp, *di, grid, s) : launch<128, false>(kp, *di, grid, s);
+}
+
+fa_status fa_fwd(const void *q, const void *k, const void *v, float *o, float *lse, int B, int H, int N, int d,
+                 int causal, float scale, void *stream) {
+    fa_fwd_params p;
+    std::memset(&p, 0, sizeof p);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.o = o;
+    p.lse = lse;
+    p.B = B;
+    p.H = H;
+    p.N = N;
+    p.d = d;
+    p.causal = causal;
+    p.scale = scale;
+    p.o_dtype = FA_O_F32;
+    return fa_fwd_ex(&p, stream);
+}
+
+fa_status fa_fwd_host(const fa_fwd_host_params *hp, void *stream) {
+    if (!hp) return FA_ERR_INVALID_ARGUMENT;
+    const fa_fwd_params *p = &hp->dev;
+    fa_status st = validate(p);
+    if (st != FA_OK) return st;
+    const size_t rows = (size_t)p->B * p->H * p->N;
+    if (rows == 0) return FA_OK;
+    if (!hp->q || !hp->k || !hp->v || !hp->o || !hp->lse) return FA_ERR_INVALID_ARGUMENT;
+    if ((hp->k_len == nullptr) != (p->k_len == nullptr)) return FA_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t in_bytes = rows * p->d * 2;
+    const size_t o_bytes = rows * p->d * (p->o_dtype == FA_O_BF16 ? 2 : 4);
+    if (cudaMemcpyAsync(const_cast<void *>(p->q), hp->q, in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(const_cast<void *>(p->k), hp->k, in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(const_cast<void *>(p->v), hp->v, in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (hp->k_len && cudaMemcpyAsync(const_cast<int32_t *>(p->k_len), hp->k_len, sizeof(int32_t) * p->B,
+                                     cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if ((st = fa_fwd_ex(p, stream)) != FA_OK) return st;
+    if (cudaMemcpyAsync(hp->o, p->o, o_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(hp->lse, p->lse, rows * sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+    if (p->dev_status) return fa_read_device_status(p->dev_status, stream);
+    return FA_OK;
+}
+
+fa_status fa_read_device_status(const int32_t *dev_status, void *stream) {
+    if (!dev_status) return FA_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    if (cudaMemcpyAsync(&h, dev_status, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+    if (h < FA_OK || h > FA_ERR_DEVICE_TIMEOUT) return FA_ERR_CUDA;
+    return (fa_status)h;
+}
+
+const char *fa_status_string(fa_status s) {
+    switch (s) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_INVALID_ARGUMENT: return "FA_ERR_INVALID_ARGUMENT";
+        case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA";
+        case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+    }
+    return "FA_ERR_UNKNOWN";
+}
+
+int fa_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,145 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact attention forward pass.
+ *
+ * The operation (page "FlashAttention (ES)", section "El problema de la
+ * atencion estandar", the Attention equation; masking from section "Fusion de
+ * operaciones en un unico kernel de CUDA"):
+ *
+ *     O   = softmax(Q K^T * scale + mask) V
+ *     lse = log( sum over allowed keys of exp(scale * q . k) )   (natural log)
+ *
+ * computed by one fused kernel launch that tiles Q, K and V through shared
+ * memory (section "Tiling y procesamiento por bloques"), keeps a running row
+ * maximum and running sum of exponentials (section "Calculo de Softmax en
+ * linea") and writes only O and lse (section "Fusion de operaciones en un
+ * unico kernel de CUDA"): no N x N buffer, no workspace of any kind.
+ *
+ * Layout (all tensors contiguous, row-major):
+ *   q, k, v : bf16  [B, H, N, d]      (one N x d matrix per (b, h))
+ *   o       : fp32  [B, H, N, d]  (fa_fwd; fa_fwd_ex may select bf16)
+ *   lse     : fp32  [B, H, N]
+ *   k_len   : int32 [B]  (fa_fwd_ex only; key j of batch b is masked iff
+ *             j >= k_len[b]; values are clamped to [0, N] on the device)
+ * Mask: causal masks key j for query i when j > i (queries and keys share
+ * positions 0..N-1).  A row with no allowed key gets O = 0, lse = -inf.
+ *
+ * Ownership: the caller owns every buffer.  The library allocates, frees and
+ * synchronises nothing (except fa_read_device_status and fa_fwd_host, which
+ * say so), holds no state beyond a per-device cache of properties and the
+ * driver's tensor-map entry point, and is safe to call from several threads.
+ *
+ * Errors: argument errors are returned synchronously and launch nothing.
+ * Device-side errors (a pipeline wait that exceeded its time limit) are
+ * written to the optional device status word.  All calls are asynchronous on
+ * `stream` (a cudaStream_t; NULL is the legacy default stream).
+ */
+#ifndef EXACT_IO_AWARE_52_FA_H
+#define EXACT_IO_AWARE_52_FA_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_EXPORT __attribute__((visibility("default")))
+#else
+#define FA_EXPORT
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARGUMENT = 1, /* NULL pointer, negative size, bad scale, bad dtype */
+    FA_ERR_MISALIGNED = 2,       /* a pointer not 16-byte aligned (TMA requirement)   */
+    FA_ERR_UNSUPPORTED = 3,      /* d not in {64, 128}, or the device is not sm_100    */
+    FA_ERR_CUDA = 4,             /* a CUDA runtime/driver call or the launch failed   */
+    FA_ERR_DEVICE_TIMEOUT = 5    /* (device status word) a pipeline wait timed out     */
+} fa_status;
+
+typedef enum { FA_O_F32 = 0, FA_O_BF16 = 1 } fa_o_dtype;
+
+/* Flags for fa_fwd_params.flags. */
+enum {
+    /* Rescale the running output whenever a row maximum grows, instead of
+     * only when it grows by more than 2^8 (the default).  Both are exact up
+     * to rounding; the default skips most rescales, this one keeps the
+     * largest softmax weight of each row at exactly 1 before rounding. */
+    FA_FLAG_EAGER_RESCALE = 1
+};
+
+/*
+ * fa_fwd -- the attention forward pass, fp32 output, no key padding.
+ *   q, k, v : device bf16 [B, H, N, d], 16-byte aligned
+ *   o       : device fp32 [B, H, N, d], 16-byte aligned
+ *   lse     : device fp32 [B, H, N]
+ *   B, H, N : >= 0 (B*H*N == 0 is a no-op returning FA_OK)
+ *   d       : 64 or 128
+ *   causal  : 0 or 1
+ *   scale   : finite, > 0 (the definition's 1/sqrt(d_k))
+ *   stream  : cudaStream_t
+ * Equivalent to fa_fwd_ex with k_len = NULL, o_dtype = FA_O_F32, flags = 0,
+ * no status word and the default time limit.
+ */
+FA_EXPORT fa_status fa_fwd(const void *q, const void *k, const void *v, float *o, float *lse,
+                 int B, int H, int N, int d, int causal, float scale, void *stream);
+
+typedef struct {
+    const void *q, *k, *v;   /* device bf16 [B, H, N, d]                              */
+    void *o;                 /* device [B, H, N, d], fp32 or bf16 per o_dtype         */
+    float *lse;              /* device fp32 [B, H, N]                                 */
+    const int32_t *k_len;    /* device int32 [B], or NULL (no key padding)           */
+    int32_t *dev_status;     /* device int32 word or NULL; the kernel stores a
+                                fa_status there on a device-side error (first error
+                                wins); the caller zeroes it before the launch        */
+    int B, H, N, d;
+    int causal;
+    float scale;
+    int o_dtype;             /* fa_o_dtype                                            */
+    int flags;               /* FA_FLAG_* bits, 0 by default                          */
+    uint32_t timeout_ms;     /* per-wait time limit on the device; 0 = 2000 ms        */
+} fa_fwd_params;
+
+/*
+ * fa_fwd_ex -- the forward pass with key padding, output dtype and a status
+ * word.  On a device-side timeout the kernel stores FA_ERR_DEVICE_TIMEOUT in
+ * *dev_status, stops, writes NaN to the rows of the tile it was working on
+ * and leaves the rows of unprocessed tiles unwritten.
+ */
+FA_EXPORT fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream);
+
+typedef struct {
+    const void *q, *k, *v;   /* host bf16 [B, H, N, d] (pinned memory for async copies) */
+    const int32_t *k_len;    /* host int32 [B] or NULL                                */
+    void *o;                 /* host output, dtype per dev.o_dtype                    */
+    float *lse;              /* host fp32 [B, H, N]                                   */
+    fa_fwd_params dev;       /* device buffers of the same shapes (q, k, v, o, lse,
+                                and k_len when k_len is not NULL) plus the options    */
+} fa_fwd_host_params;
+
+/*
+ * fa_fwd_host -- end-to-end call on HOST buffers: copies q, k, v (and k_len)
+ * host -> device into the caller's device buffers, runs fa_fwd_ex, copies o
+ * and lse device -> host, and synchronises `stream` before returning.
+ * One cudaMemcpyAsync per buffer.  If dev.dev_status is set, a device-side
+ * error found after the copies is returned as its fa_status.
+ */
+FA_EXPORT fa_status fa_fwd_host(const fa_fwd_host_params *p, void *stream);
+
+/*
+ * fa_read_device_status -- synchronises `stream`, reads the device status
+ * word and returns it as a fa_status (FA_ERR_CUDA if the read fails).
+ */
+FA_EXPORT fa_status fa_read_device_status(const int32_t *dev_status, void *stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FA_EXPORT const char *fa_status_string(fa_status s);
+
+/* Library version as an integer MAJOR*10000 + MINOR*100 + PATCH. */
+FA_EXPORT int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_IO_AWARE_52_FA_H */

@@ -1,0 +1,51 @@
+/*
+ * fa_selftest.h -- single-CTA checks of the sm_100a building blocks of the
+ * attention kernel (libfa_selftest.so).  Each call launches one small kernel
+ * on `stream` (a cudaStream_t), synchronises it and returns 0 on success, 1 on
+ * a bad argument, 4 on a CUDA error.  Device-side time-outs store 5 in
+ * *status (caller-zeroed device int32).  All pointers are device pointers,
+ * 16-byte aligned, owned by the caller.
+ *
+ * These exercise the tiling step of the page "FlashAttention (ES)", section
+ * "Tiling y procesamiento por bloques" (TMA into shared memory), and the two
+ * matrix products of section "Fusion de operaciones en un unico kernel de
+ * CUDA" (Q K^T and the product with V) on the tensor cores.
+ */
+#ifndef EXACT_IO_AWARE_52_FA_SELFTEST_H
+#define EXACT_IO_AWARE_52_FA_SELFTEST_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_SELFTEST_EXPORT __attribute__((visibility("default")))
+#else
+#define FA_SELFTEST_EXPORT
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* TMA-load the bf16 tile src[128][64] with 128-byte swizzle and copy the raw
+ * 16384-byte shared-memory image to dst. */
+FA_SELFTEST_EXPORT int fa_selftest_tma_sw128(const void *src, void *dst, int32_t *status, void *stream);
+
+/* s[128][128] (fp32) = a[128][K] * b[128][K]^T with tcgen05.mma, a and b bf16
+ * K-major in shared memory; K in {64, 128}. */
+FA_SELFTEST_EXPORT int fa_selftest_mma_ss(const void *a, const void *b, float *s, int K, int32_t *status,
+                                          void *stream);
+
+/* o[128][D] (fp32) = p[128][128] * v[128][D] with tcgen05.mma, p (bf16) staged
+ * in tensor memory, v (bf16) MN-major in shared memory; D in {64, 128}. */
+FA_SELFTEST_EXPORT int fa_selftest_mma_ts(const void *p, const void *v, float *o, int D, int32_t *status,
+                                          void *stream);
+
+/* Wait on a barrier nothing arrives at, with a limit of timeout_ms; the wait
+ * must give up and store 5 in *status. */
+FA_SELFTEST_EXPORT int fa_selftest_wait_timeout(int32_t *status, uint32_t timeout_ms, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_IO_AWARE_52_FA_SELFTEST_H */

@@ -1,0 +1,219 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Tolerances for bf16 inputs with fp32 accumulation: max |dO| <= 1e-2,
+mean |dO| <= 1e-3, max |dlse| / max(|lse|, 1) <= 1e-4 (tests/gpu_util.py).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_52_b200 import _binding as fb
+from exact_io_aware_52_b200 import workloads
+from tests.gpu_util import check_case, check_workload, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def rand_inputs(B, H, N, d, seed, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    q = (torch.randn(B, H, N, d, generator=g) * std).to(torch.bfloat16)
+    k = (torch.randn(B, H, N, d, generator=g) * std).to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+# ------------------------------------------------------------ the five workloads
+@pytest.mark.parametrize("wid", [1, 2, 3, 4, 5])
+def test_workload_parity(wid):
+    """Each seeded workload at its full size, in the launch configuration the
+    benchmark times (all rows for 1-3, the seeded row sample for 4-5)."""
+    stats = check_workload(workloads.WORKLOADS[wid])
+    print(f"workload {wid}: {stats}")
+
+
+# ------------------------------------------------------------ shapes and tails
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 7, 127, 128, 129, 200, 383, 640])
+def test_ragged_shapes(N, d, causal):
+    """Tiles with ragged tails in both the query and the key direction."""
+    q, k, v = rand_inputs(2, 3, N, d, seed=1000 + N * 7 + d + causal)
+    check_case(q, k, v, causal, 1.0 / math.sqrt(d))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_more_units_than_sms(d):
+    """B*H*ceil(N/128) well above the SM count: each persistent CTA walks
+    several work units (and both walking directions of the schedule)."""
+    q, k, v = rand_inputs(4, 100, 257, d, seed=77 + d)
+    for causal in (False, True):
+        check_case(q, k, v, causal, 1.0 / math.sqrt(d))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_padding_edges(d, causal):
+    """Key lengths 0 (no allowed key: O = 0, lse = -inf), 1, N-1, N, beyond N
+    (clamped) and negative (clamped to 0), mixed in one batch."""
+    N = 300
+    k_len = [0, 1, N - 1, N, N + 50, -5, 128, 129]
+    q, k, v = rand_inputs(len(k_len), 2, N, d, seed=31 + d + causal)
+    check_case(q, k, v, causal, 1.0 / math.sqrt(d), k_len=k_len)
+
+
+# ------------------------------------------------------------ closed forms on the GPU
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_gives_means(causal):
+    """Q = 0: O_i is the mean of the allowed V rows, lse_i = ln(#allowed)."""
+    B, H, N, d = 1, 2, 333, 128
+    g = torch.Generator().manual_seed(5)
+    q = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+    k = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    o, lse = run_gpu(q, k, v, causal, 0.1)
+    vv = v.double()
+    if causal:
+        ref = vv.cumsum(2) / torch.arange(1, N + 1, dtype=torch.float64).view(1, 1, N, 1)
+        lse_ref = torch.log(torch.arange(1, N + 1, dtype=torch.float64)).expand(B, H, N)
+    else:
+        ref = vv.mean(2, keepdim=True).expand(B, H, N, d)
+        lse_ref = torch.full((B, H, N), math.log(N), dtype=torch.float64)
+    assert (o.double() - ref).abs().max().item() < 1e-2
+    assert (lse.double() - lse_ref).abs().max().item() < 1e-4 * max(1.0, math.log(N))
+
+
+def test_dominant_key_selects_its_value():
+    """Key 300 scores 40 above every other key for every query (q = 8 e_0,
+    k_300 = 5 e_0, other keys 0), so each output row is V_300 to within
+    511 e^-40 of weight."""
+    B, H, N, d = 1, 1, 512, 64
+    g = torch.Generator().manual_seed(6)
+    q = torch.zeros(B, H, N, d)
+    k = torch.zeros(B, H, N, d)
+    q[..., 0] = 8.0
+    k[0, 0, :, 1] = 1.0
+    k[0, 0, 300, 0] = 5.0
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    o, _ = run_gpu(q, k, v, False, 1.0)
+    ref = v[0, 0, 300].double().expand(N, d)
+    assert (o[0, 0].double() - ref).abs().max().item() < 1e-2
+
+
+# ------------------------------------------------------------ adversarial inputs
+def test_monotone_logits_force_rescale_every_tile():
+    """Scores that grow along the keys move the row maximum on every tile."""
+    B, H, N, d = 1, 2, 1024, 64
+    q = torch.zeros(B, H, N, d)
+    k = torch.zeros(B, H, N, d)
+    q[..., 0] = 1.0
+    k[..., 0] = torch.linspace(-20, 60, N)
+    g = torch.Generator().manual_seed(8)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    for flags in (0, fb.FA_FLAG_EAGER_RESCALE):
+        for causal in (False, True):
+            check_case(q.to(torch.bfloat16), k.to(torch.bfloat16), v, causal, 1.0, flags=flags)
+
+
+def test_max_key_in_last_tile():
+    B, H, N, d = 1, 1, 900, 128
+    q, k, v = rand_inputs(B, H, N, d, seed=9)
+    k[0, 0, N - 1] = (q[0, 0].float().mean(0) * 6).to(torch.bfloat16)
+    check_case(q, k, v, False, 1.0 / math.sqrt(d))
+
+
+def test_all_equal_logits():
+    B, H, N, d = 2, 2, 700, 64
+    g = torch.Generator().manual_seed(10)
+    q = torch.ones(B, H, N, d).to(torch.bfloat16)
+    k = torch.ones(B, H, N, d).to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    for causal in (False, True):
+        check_case(q, k, v, causal, 0.125)
+
+
+@pytest.mark.parametrize("std", [4.0, 8.0])
+@pytest.mark.parametrize("flags", [0, fb.FA_FLAG_EAGER_RESCALE])
+def test_large_logits(std, flags):
+    """N(0, 4^2) and N(0, 8^2) queries and keys: near one-hot softmax rows."""
+    q, k, v = rand_inputs(1, 4, 2048, 128, seed=int(std) * 11 + flags, std=std)
+    check_case(q, k, v, True, 1.0 / math.sqrt(128), flags=flags)
+
+
+# ------------------------------------------------------------ options and API paths
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_output(d):
+    """bf16 O: its rounding (2^-9 relative) is added to the error budget."""
+    q, k, v = rand_inputs(2, 4, 555, d, seed=12 + d)
+    check_case(q, k, v, True, 1.0 / math.sqrt(d), out_dtype=torch.bfloat16, tol_max=2e-2, tol_mean=2e-3)
+
+
+def test_deterministic():
+    q, k, v = rand_inputs(2, 8, 1000, 128, seed=13)
+    o1, l1 = run_gpu(q, k, v, True, 0.088)
+    o2, l2 = run_gpu(q, k, v, True, 0.088)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_side_stream_and_fa_fwd():
+    """fa_fwd (fp32, no padding) on a non-default stream equals fa_fwd_ex."""
+    q, k, v = rand_inputs(1, 4, 384, 64, seed=14)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty(1, 4, 384, 64, device=dev)
+    lse = torch.empty(1, 4, 384, device=dev)
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        fb.fa_fwd(qd, kd, vd, o, lse, True, 0.125, stream=s)
+    s.synchronize()
+    o2, l2 = run_gpu(q, k, v, True, 0.125)
+    assert torch.equal(o.cpu(), o2) and torch.equal(lse.cpu(), l2)
+
+
+def test_host_entry_point():
+    """fa_fwd_host: pinned host buffers in and out, copies inside the call."""
+    B, H, N, d = 2, 3, 260, 128
+    q, k, v = rand_inputs(B, H, N, d, seed=15)
+    dev = torch.device("cuda:0")
+    k_len = torch.tensor([200, 260], dtype=torch.int32)
+    qh, kh, vh, klh = q.pin_memory(), k.pin_memory(), v.pin_memory(), k_len.pin_memory()
+    oh = torch.empty(B, H, N, d).pin_memory()
+    lh = torch.empty(B, H, N).pin_memory()
+    qd, kd, vd = (torch.empty_like(t, device=dev) for t in (q, k, v))
+    kld = torch.empty(B, dtype=torch.int32, device=dev)
+    od = torch.empty(B, H, N, d, device=dev)
+    ld = torch.empty(B, H, N, device=dev)
+    fb.fa_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, True, 1 / math.sqrt(d), k_len_h=klh, k_len_d=kld)
+    o2, l2 = run_gpu(q, k, v, True, 1 / math.sqrt(d), k_len=[200, 260])
+    assert torch.equal(oh, o2) and torch.equal(lh, l2)
+
+
+def test_no_device_memory_allocated():
+    """The library allocates nothing: free device memory is unchanged across
+    a launch (O(N) memory, no N x N buffer, no workspace)."""
+    dev = torch.device("cuda:0")
+    q, k, v = rand_inputs(1, 8, 4096, 128, seed=16)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty(1, 8, 4096, 128, device=dev)
+    lse = torch.empty(1, 8, 4096, device=dev)
+    fb.fa_fwd(qd, kd, vd, o, lse, True, 0.088)  # first call: module load, attributes
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        fb.fa_fwd(qd, kd, vd, o, lse, True, 0.088)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free0 == free1
+
+
+def test_status_word_stays_clear():
+    q, k, v = rand_inputs(1, 2, 256, 64, seed=17)
+    dev = torch.device("cuda:0")
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    o = torch.empty(1, 2, 256, 64, device=dev)
+    lse = torch.empty(1, 2, 256, device=dev)
+    fb.fa_fwd_ex(q.to(dev), k.to(dev), v.to(dev), o, lse, False, 0.125, dev_status=st, timeout_ms=500)
+    assert fb.read_device_status(st) == fb.FA_OK

@@ -1,0 +1,90 @@
+"""GPU checks of the sm_100a building blocks, one at a time, through the
+self-test C ABI (include/fa_selftest.h)."""
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_52_b200 import _binding as fb
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev():
+    return torch.device("cuda:0")
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device=_dev())
+
+
+def _p(t):
+    return t.data_ptr()
+
+
+def test_tma_128b_swizzle_image():
+    """A 128x64 bf16 box lands in shared memory with the 128-byte swizzle:
+    16-byte chunk c of row r sits at chunk position c xor (r mod 8)."""
+    lib = fb.load_selftest()
+    src = torch.arange(128 * 64, dtype=torch.int32).reshape(128, 64)
+    src_bits = (src & 0x7FFF).to(torch.int16)  # distinct 16-bit patterns per element
+    src_d = src_bits.view(torch.bfloat16).to(_dev())
+    dst = torch.zeros(16384, dtype=torch.uint8, device=_dev())
+    st = _status()
+    assert lib.fa_selftest_tma_sw128(_p(src_d), _p(dst), _p(st), None) == 0
+    assert st.item() == 0
+    img = dst.cpu().numpy().view(np.int16)
+    expect = np.zeros(128 * 64, dtype=np.int16)
+    s = src_bits.numpy()
+    for r in range(128):
+        for c in range(64):
+            chunk, within = divmod(c, 8)
+            pos = r * 64 + ((chunk ^ (r % 8)) * 8) + within
+            expect[pos] = s[r, c]
+    np.testing.assert_array_equal(img, expect)
+
+
+@pytest.mark.parametrize("K", [64, 128])
+def test_tcgen05_ss_matches_matmul(K):
+    """S = A B^T on the tensor cores (both operands K-major, 128-byte swizzle)
+    equals the float64 product of the same bf16 values to fp32 accuracy."""
+    lib = fb.load_selftest()
+    g = torch.Generator().manual_seed(100 + K)
+    a = torch.randn(128, K, generator=g).to(torch.bfloat16)
+    b = torch.randn(128, K, generator=g).to(torch.bfloat16)
+    s = torch.full((128, 128), float("nan"), device=_dev())
+    st = _status()
+    assert lib.fa_selftest_mma_ss(_p(a.to(_dev())), _p(b.to(_dev())), _p(s), K, _p(st), None) == 0
+    assert st.item() == 0
+    ref = a.double() @ b.double().T
+    np.testing.assert_allclose(s.cpu().double().numpy(), ref.numpy(), rtol=0, atol=2e-4)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_tcgen05_ts_matches_matmul(D):
+    """O = P V with P staged in tensor memory (two bf16 per column) and V
+    MN-major in shared memory equals the float64 product."""
+    lib = fb.load_selftest()
+    g = torch.Generator().manual_seed(200 + D)
+    p = torch.rand(128, 128, generator=g).to(torch.bfloat16)
+    v = torch.randn(128, D, generator=g).to(torch.bfloat16)
+    o = torch.full((128, D), float("nan"), device=_dev())
+    st = _status()
+    assert lib.fa_selftest_mma_ts(_p(p.to(_dev())), _p(v.to(_dev())), _p(o), D, _p(st), None) == 0
+    assert st.item() == 0
+    ref = p.double() @ v.double()
+    np.testing.assert_allclose(o.cpu().double().numpy(), ref.numpy(), rtol=0, atol=2e-4)
+
+
+def test_bounded_wait_gives_up():
+    """A wait on a barrier nothing arrives at gives up after its limit,
+    reports FA_ERR_DEVICE_TIMEOUT, and the context stays usable."""
+    import time
+    lib = fb.load_selftest()
+    st = _status()
+    t0 = time.time()
+    assert lib.fa_selftest_wait_timeout(_p(st), 200, None) == 0
+    dt = time.time() - t0
+    assert st.item() == fb.FA_ERR_DEVICE_TIMEOUT
+    assert dt < 5.0
+    x = torch.ones(16, device=_dev())
+    assert float((x * 2).sum().item()) == 32.0

@@ -48,7 +48,7 @@ KERNEL_SOURCES = ["fa_fwd_kernel.cuh", "sm100_ptx.cuh", "fa_api.cu"]
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -113,9 +113,9 @@ class ClockSampler:
         self.proc = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
         props = torch.cuda.get_device_properties(device_index)
-        self.bus = None
+        self.bus = None  # "BB:DD" (bus:device, hex) of the GPU this rank uses
         try:
-            self.bus = "%08X:%02X:%02X" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            self.bus = "%02X:%02X" % (props.pci_bus_id, props.pci_device_id)
         except AttributeError:
             pass
 
@@ -146,7 +146,8 @@ class ClockSampler:
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) != len(self.FIELDS):
                     continue
-                if self.bus and not parts[0].upper().endswith(self.bus[-7:]):
+                bus_dev = ":".join(parts[0].upper().split(".")[0].split(":")[-2:])
+                if self.bus and bus_dev != self.bus:
                     continue
                 rows.append(parts)
         if not rows:

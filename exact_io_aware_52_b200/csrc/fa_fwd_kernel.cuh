@@ -203,7 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
             }
 
             float m_ref = 0.f;  // reference maximum, log2 units
-            float l = 0.f;      // running sum of 2^(x - m_ref)
+            float l = 0.f;      // running sum of 2^(x - m_ref), unrounded: gives lse
+            float lr = 0.f;     // running sum of bf16(2^(x - m_ref)), the weights the tensor core
+                                // multiplies V by: dividing O by it makes O an exact convex
+                                // combination of V rows (a lone dominant weight is not rounded away)
             for (int j = 0; j < tc.n_kv; ++j, ++g) {
                 const uint32_t buf = g & 1;
                 ok = mbar_wait(&bars[C::kBarSFull + buf], (g >> 1) & 1, abort_flag, p.timeout_ns);
@@ -251,16 +254,18 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
                 if (j == 0) {
                     m_ref = (m_new == NEG_INF) ? 0.f : m_new;
                     l = 0.f;
+                    lr = 0.f;
                 } else if (m_new > m_ref + p.tau) {
                     alpha = ex2_approx(m_ref - m_new);
                     l *= alpha;
+                    lr *= alpha;
                     m_ref = m_new;
                     resc = true;
                 }
                 const float neg_m = -m_ref;
-                float ls[8];
+                float ls[8], lrs[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) ls[i] = 0.f;
+                for (int i = 0; i < 8; ++i) ls[i] = lrs[i] = 0.f;
                 uint32_t pk0[32], pk1[32];  // keys [0,64) and [64,128), two bf16 per column
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
@@ -268,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
                     const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, neg_m));
                     ls[(c >> 1) & 7] += p0 + p1;
                     pk0[c >> 1] = pack_bf16x2(p0, p1);
+                    lrs[(c >> 1) & 7] += bf16x2_lo(pk0[c >> 1]) + bf16x2_hi(pk0[c >> 1]);
                 }
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
@@ -275,8 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
                     const float p1 = ex2_approx(fmaf(s[64 + c + 1], p.scale_log2, neg_m));
                     ls[(c >> 1) & 7] += p0 + p1;
                     pk1[c >> 1] = pack_bf16x2(p0, p1);
+                    lrs[(c >> 1) & 7] += bf16x2_lo(pk1[c >> 1]) + bf16x2_hi(pk1[c >> 1]);
                 }
                 l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                lr += ((lrs[0] + lrs[1]) + (lrs[2] + lrs[3])) + ((lrs[4] + lrs[5]) + (lrs[6] + lrs[7]));
                 {
                     const uint32_t a = tmem + lane_off + col_p(buf);
                     tmem_st32(a + 0, pk0);
@@ -325,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
                 break;
             }
             tc_fence_after();
-            const float inv_l = 1.f / l;
+            const float inv_l = 1.f / lr;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t r[32];

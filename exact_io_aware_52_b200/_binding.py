@@ -98,6 +98,8 @@ def load_selftest():
             lib.fa_selftest_mma_ss.argtypes = [vp, vp, vp, i, vp, vp]
             lib.fa_selftest_mma_ts.restype = i
             lib.fa_selftest_mma_ts.argtypes = [vp, vp, vp, i, vp, vp]
+            lib.fa_selftest_exp2_poly.restype = i
+            lib.fa_selftest_exp2_poly.argtypes = [vp, vp, i, vp]
             lib.fa_selftest_wait_timeout.restype = i
             lib.fa_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
             _selftest = lib

@@ -90,7 +90,7 @@ fa_status validate(const fa_fwd_params *p) {
     if (p->d != 64 && p->d != 128) return FA_ERR_UNSUPPORTED;
     const long long rows = (long long)p->B * p->H * p->N;
     if (rows == 0) return FA_OK;
-    if ((long long)p->B * p->H > 0x7fffffffLL || (long long)p->B * p->H * ((p->N + 127) / 128) > 0x7fffffffLL)
+    if ((long long)p->B * p->H > 0x7fffffffLL || (long long)p->B * p->H * ((p->N + 255) / 256) > 0x7fffffffLL)
         return FA_ERR_INVALID_ARGUMENT;
     if (!p->q || !p->k || !p->v || !p->o || !p->lse) return FA_ERR_INVALID_ARGUMENT;
     if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v) || !aligned16(p->o)) return FA_ERR_MISALIGNED;
@@ -148,14 +148,14 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     kp.B = p->B;
     kp.H = p->H;
     kp.N = p->N;
-    kp.n_qtiles = (p->N + fa::BM - 1) / fa::BM;
-    kp.n_tiles = BH * kp.n_qtiles;
+    kp.n_blocks = (p->N + fa::kUnitRows - 1) / fa::kUnitRows;
+    kp.n_units = BH * kp.n_blocks;
     kp.causal = p->causal;
     kp.scale_log2 = (float)((double)p->scale * 1.4426950408889634074);
     kp.tau = (p->flags & FA_FLAG_EAGER_RESCALE) ? 0.f : 8.f;
     kp.timeout_ns = (uint64_t)(p->timeout_ms ? p->timeout_ms : 2000u) * 1000000ull;
 
-    const int grid = kp.n_tiles < di->num_sms ? kp.n_tiles : di->num_sms;
+    const int grid = kp.n_units < di->num_sms ? kp.n_units : di->num_sms;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = p->o_dtype == FA_O_BF16;
     if (p->d == 64) return bf16 ? launch<64, true>(kp, *di, grid, s) : launch<64, false>(kp, *di, grid, s);

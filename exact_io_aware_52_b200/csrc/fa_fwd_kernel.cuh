@@ -5,32 +5,41 @@
 // estandar"), following the three techniques of section "Innovaciones clave de
 // FlashAttention":
 //   * tiling ("Tiling y procesamiento por bloques"): a work unit is one
-//     128-row query tile of one (b, h); its 128-key K and V tiles stream from
-//     HBM into shared memory through TMA and a multi-stage mbarrier ring, and
-//     the score tile S = Q K_j^T never leaves the SM;
+//     256-row query block of one (b, h), split into two 128-row tiles A and
+//     B; the 128-key K and V tiles stream from HBM into shared memory through
+//     TMA and mbarrier rings and each feeds both query tiles; the score tile
+//     S = Q K_j^T never leaves the SM;
 //   * online softmax ("Calculo de Softmax en linea"): each row keeps a
-//     reference maximum m and a running sum l of exp2 terms; a new tile's
+//     reference maximum m and two running sums of exp2 terms; a new tile's
 //     terms are taken relative to m, and when m must grow the accumulated
-//     output and l are multiplied by 2^(m_old - m_new);
+//     output and sums are multiplied by 2^(m_old - m_new);
 //   * one fused kernel ("Fusion de operaciones en un unico kernel de CUDA"):
 //     Q K^T, masking, softmax and the product with V run in this one kernel,
 //     which writes only O and lse.
 //
-// Blackwell mapping (one CTA per SM, persistent over work units):
-//   warps 0-3  softmax: thread t owns query row t of the tile; reads its S row
-//              from tensor memory (TMEM), masks, updates m and l, writes the
-//              bf16 probabilities P back to TMEM, rescales O in TMEM when
-//              needed, and runs the epilogue (O / l, lse) for its row;
-//   warp 4     MMA issuer (one thread): S_j = Q K_j^T (A and B from shared
-//              memory) and O += P_j V_j (A = P from TMEM, B = V_j from shared
-//              memory) with tcgen05.mma, fp32 accumulation in TMEM;
-//   warp 5     TMA producer (one thread): Q once per work unit, K_j and V_j
-//              through the stage ring.
-// TMEM (512 columns): S double buffer [0,256), O [256, 256+D), P double
-// buffer [384, 512) (128 bf16 keys pack into 64 columns).
-// The MMA issue order is Q K_g^T, then P_{g-1} V_{g-1}, over a global sequence
-// g of key tiles that runs across work units, so the tensor core computes the
-// next score tile while the softmax warps work on the current one.
+// Blackwell mapping (one CTA per SM, persistent over work units), 12 warps:
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread t of a
+//              warpgroup owns row t of its tile; it reads its S row from
+//              tensor memory (TMEM), masks, updates m and the sums, writes the
+//              bf16 probabilities P back over the S row in TMEM, rescales its
+//              O row in TMEM when m moved, and runs the epilogue for its row;
+//   warp 8     MMA issuer (one thread): S_X = Q_X K_j^T (both operands in
+//              shared memory) and O_X += P_X V_j (P from TMEM, V_j from shared
+//              memory), tcgen05.mma with fp32 accumulation in TMEM;
+//   warp 9     TMA producer (one thread): Q_A and Q_B once per unit, K_j and
+//              V_j through separate rings (warps 10-11 idle).
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256, 256+D),
+// O_B [256+D, 256+2D); P_X occupies the first 64 columns of S_X (two bf16 per
+// 32-bit column).
+//
+// MMA issue order inside a unit, for key tiles j = 1, 2, ...:
+//     P_A V_{j-1},  Q_A K_j^T,  P_B V_{j-1},  Q_B K_j^T
+// so the tensor core works on one tile while the other tile's softmax runs.
+// tcgen05.mma operations issued by one thread execute in issue order, which
+// makes two things safe: Q_X K_j^T overwrites the S_X columns holding P_X only
+// after P_X V_{j-1} has read them, and the commit that signals "S_X(j) ready"
+// also covers P_X V_{j-1}, so the softmax may rescale O_X as soon as S_X(j)
+// arrives.
 //
 // Every wait is bounded in wall time.  On time-out the CTA raises a shared
 // abort flag, records FA_ERR_DEVICE_TIMEOUT in the optional status word,
@@ -41,17 +50,36 @@
 
 namespace fa {
 
-constexpr int BM = 128;  // query rows per tile (tcgen05 M)
-constexpr int BN = 128;  // keys per tile
-constexpr int kSoftmaxWarps = 4;
-constexpr int kMmaWarp = 4;
-constexpr int kLoadWarp = 5;
-constexpr int kThreads = 192;
+constexpr int BM = 128;        // query rows per tile (tcgen05 M)
+constexpr int BN = 128;        // keys per tile
+constexpr int kQTiles = 2;     // query tiles per work unit
+constexpr int kUnitRows = BM * kQTiles;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;   // warps 10-11 only complete the third warpgroup
+constexpr int kThreads = 384;
+// Register split (setmaxnreg): the launch gives 384 x 168; the two softmax
+// warpgroups take 216 each and the MMA/TMA warpgroup keeps 72:
+// 256 * 216 + 128 * 72 = 64512 = 384 * 168, and 216 + 216 + 72 <= 512 per lane
+// on every SM sub-partition (one warp of each warpgroup per sub-partition).
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;
-__device__ __forceinline__ uint32_t col_s(uint32_t buf) { return buf * 128u; }        // S double buffer
-__device__ __forceinline__ uint32_t col_p(uint32_t buf) { return 384u + buf * 64u; }  // P double buffer
 constexpr int kStatusTimeout = 5;  // FA_ERR_DEVICE_TIMEOUT
+// Of every kPolyPeriod key pairs of a score row, the last kPolyPairs take
+// their exponentials from the FMA-pipe polynomial, the rest from MUFU ex2.
+// Measured on workload 4 (B200, 300 launches): 0 of 4 -> 2.30 ms, 1 of 4 ->
+// 2.44 ms, 2 of 4 -> 2.49 ms: the softmax is not MUFU-throughput bound here,
+// so the polynomial's extra instructions only cost; it stays off.
+constexpr int kPolyPeriod = 4;
+constexpr int kPolyPairs = 0;
+// P to bf16: round to nearest even (cvt) when false; truncation (keep the
+// high half of each fp32 word, one byte permute per pair) when true.
+constexpr bool kPackTruncate = false;
+
+__device__ __forceinline__ uint32_t col_s(uint32_t x) { return x * 128u; }                  // S_X, P_X
+__device__ __forceinline__ uint32_t col_o(uint32_t x, uint32_t d) { return 256u + x * d; }  // O_X
 
 struct FwdParams {
     CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps over [B*H][N][D] bf16; box {64, 128, 1}; 128-byte swizzle
@@ -60,8 +88,8 @@ struct FwdParams {
     const int32_t *k_len;          // [B] or nullptr
     int32_t *status;               // device status word or nullptr
     int B, H, N;
-    int n_qtiles;                  // ceil(N / BM)
-    int n_tiles;                   // B * H * n_qtiles
+    int n_blocks;                  // ceil(N / 256)
+    int n_units;                   // B * H * n_blocks
     int causal;
     float scale_log2;              // scale * log2(e)
     float tau;                     // rescale threshold in log2 units (<= 0: rescale on any growth)
@@ -73,23 +101,24 @@ struct Cfg {
     static constexpr int kChunks = D / 64;          // 64-element (128-byte) column blocks per row
     static constexpr int kChunkBytes = BM * 128;    // one column block of a 128-row tile
     static constexpr int kTileBytes = BM * D * 2;   // one 128 x D bf16 tile
-    static constexpr int kStages = (D == 128) ? 3 : 4;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTileBytes;
-    static constexpr int kOffV = kOffK + kStages * kTileBytes;
-    static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+    static constexpr int kKStages = (D == 128) ? 3 : 4;
+    static constexpr int kVStages = (D == 128) ? 2 : 4;
+    static constexpr int kOffQ = 0;                                   // Q_A, Q_B
+    static constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
+    static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+    static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
     // barrier slots
     static constexpr int kBarQFull = 0;
     static constexpr int kBarQEmpty = 1;
     static constexpr int kBarKFull = 2;
-    static constexpr int kBarVFull = kBarKFull + kStages;
-    static constexpr int kBarKVEmpty = kBarVFull + kStages;
-    static constexpr int kBarSFull = kBarKVEmpty + kStages;  // 2
-    static constexpr int kBarPFull = kBarSFull + 2;          // 2
-    static constexpr int kBarODone = kBarPFull + 2;
-    static constexpr int kBarOFinal = kBarODone + 1;
-    static constexpr int kBarOFree = kBarOFinal + 1;
-    static constexpr int kBarDrain = kBarOFree + 1;
+    static constexpr int kBarKEmpty = kBarKFull + kKStages;
+    static constexpr int kBarVFull = kBarKEmpty + kKStages;
+    static constexpr int kBarVEmpty = kBarVFull + kVStages;
+    static constexpr int kBarSFull = kBarVEmpty + kVStages;  // [2], per query tile
+    static constexpr int kBarPFull = kBarSFull + 2;          // [2]
+    static constexpr int kBarOFinal = kBarPFull + 2;         // [2]
+    static constexpr int kBarOFree = kBarOFinal + 2;         // [2]
+    static constexpr int kBarDrain = kBarOFree + 2;
     static constexpr int kNumBars = kBarDrain + 1;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 4;
@@ -97,10 +126,13 @@ struct Cfg {
     static constexpr int kSmemBytes = kSmemUsed + 1024;  // + slack to align the base to 1024 bytes
     static_assert(kChunkBytes % 1024 == 0 && kTileBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
+    static_assert(2 * kSmemBytes > 233472, "one CTA per SM: TMEM is allocated whole");
 };
 
-struct TileCoord {
-    int bh, b, qt, n_kv;
+struct UnitCoord {
+    int bh, b, blk;
+    int n[2];  // key tiles of query tile A and B (a prefix [0, n) of the key tiles)
+    int nmax;
 };
 
 // Work unit k of this CTA: bands of gridDim.x consecutive units, walked in
@@ -111,17 +143,23 @@ __device__ __forceinline__ int unit_index(int k) {
     return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-__device__ __forceinline__ TileCoord decode_tile(const FwdParams &p, int t) {
-    TileCoord tc;
+__device__ __forceinline__ UnitCoord decode_unit(const FwdParams &p, int t) {
+    UnitCoord u;
     const int BH = p.B * p.H;
-    tc.qt = p.n_qtiles - 1 - t / BH;  // longest (causal) query tiles first
-    tc.bh = t % BH;
-    tc.b = tc.bh / p.H;
-    int kv_end = p.N;
-    if (p.k_len) kv_end = min(max(__ldg(p.k_len + tc.b), 0), p.N);
-    if (p.causal) kv_end = min(kv_end, (tc.qt + 1) * BM);
-    tc.n_kv = (kv_end + BN - 1) / BN;
-    return tc;
+    u.blk = p.n_blocks - 1 - t / BH;  // longest (causal) query blocks first
+    u.bh = t % BH;
+    u.b = u.bh / p.H;
+    int kv_lim = p.N;
+    if (p.k_len) kv_lim = min(max(__ldg(p.k_len + u.b), 0), p.N);
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        const int first = u.blk * kUnitRows + x * BM;
+        int e = kv_lim;
+        if (p.causal) e = min(e, first + BM);
+        u.n[x] = (first < p.N) ? (e + BN - 1) / BN : 0;
+    }
+    u.nmax = max(u.n[0], u.n[1]);
+    return u;
 }
 
 __device__ __forceinline__ void record_timeout(const FwdParams &p) {
@@ -132,6 +170,408 @@ __device__ __forceinline__ void record_timeout(const FwdParams &p) {
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t timeout_ns) {
     int dummy = 0;
     return mbar_wait(bar, parity, &dummy, timeout_ns);
+}
+
+template <int D, bool O_BF16>
+__device__ __forceinline__ void store_row_chunk(void *o, size_t row_id, int ch, const uint32_t (&r)[32], float inv_l) {
+    if constexpr (O_BF16) {
+        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(o) + row_id * D + ch * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l);
+            dst[i] = v;
+        }
+    } else {
+        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(o) + row_id * D + ch * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(r[4 * i + 0]) * inv_l, __uint_as_float(r[4 * i + 1]) * inv_l,
+                                 __uint_as_float(r[4 * i + 2]) * inv_l, __uint_as_float(r[4 * i + 3]) * inv_l);
+    }
+}
+
+// Fills one output row with a constant (0 for rows without allowed keys, NaN
+// for rows of a unit abandoned after a time-out) and sets its lse.
+template <int D, bool O_BF16>
+__device__ __forceinline__ void fill_row(void *o, float *lse, size_t row_id, bool nan, float lv) {
+    if constexpr (O_BF16) {
+        const uint16_t b = nan ? 0x7fc0 : 0;
+        uint16_t *dst = reinterpret_cast<uint16_t *>(o) + row_id * D;
+        for (int i = 0; i < D; ++i) dst[i] = b;
+    } else {
+        const float f = nan ? __int_as_float(0x7fc00000) : 0.f;
+        float *dst = reinterpret_cast<float *>(o) + row_id * D;
+        for (int i = 0; i < D; ++i) dst[i] = f;
+    }
+    lse[row_id] = lv;
+}
+
+// max of 64 scores: four chains of three-input maxima
+__device__ __forceinline__ float max64(const float *v) {
+    float a0 = fmaxf(v[0], v[1]), a1 = fmaxf(v[2], v[3]), a2 = fmaxf(v[4], v[5]), a3 = fmaxf(v[6], v[7]);
+#pragma unroll
+    for (int c = 8; c < 64; c += 8) {
+        a0 = fmax3(a0, v[c], v[c + 1]);
+        a1 = fmax3(a1, v[c + 2], v[c + 3]);
+        a2 = fmax3(a2, v[c + 4], v[c + 5]);
+        a3 = fmax3(a3, v[c + 6], v[c + 7]);
+    }
+    return fmaxf(fmax3(a0, a1, a2), a3);
+}
+
+// Scores of keys [64H, 64H+64) of this thread's row: two 32-column TMEM loads.
+template <int H>
+__device__ __forceinline__ void load_scores(uint32_t t_s, float *s) {
+    tmem_ld32f(t_s + 64 * H, s + 64 * H);
+    tmem_ld32f(t_s + 64 * H + 32, s + 64 * H + 32);
+    tmem_ld_wait();
+    tmem_reg_fence_f<64>(s + 64 * H);
+}
+
+// Masking step for keys [64H, 64H+64) of a tile starting at key kv0: keys at
+// or beyond the row's limit get -inf.
+template <int H>
+__device__ __forceinline__ void mask_scores(float *s, int kv0, int lim) {
+#pragma unroll
+    for (int c = 64 * H; c < 64 * H + 64; ++c)
+        if (kv0 + c >= lim) s[c] = __int_as_float(0xff800000);
+}
+
+// Probabilities of keys [64H, 64H+64) of one score row against reference -neg_m
+// (log2 units): p = 2^(s * scale_log2 - m), summed unrounded into `ls` and as
+// the bf16 values the tensor core will use into `lrs`, and packed as bf16
+// pairs into pk (column c holds keys 64H + 2c and 64H + 2c + 1).
+template <int H>
+__device__ __forceinline__ void exp_half(const float *s, float scale_log2, float neg_m, uint32_t (&pk)[32],
+                                         float2 &ls, float &lrs) {
+    const float2 sl2 = make_float2(scale_log2, scale_log2);
+    const float2 nm = make_float2(neg_m, neg_m);
+    float2 a[4] = {ls, make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float b[4] = {lrs, 0.f, 0.f, 0.f};
+    float2 b2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+        const float2 xx = __ffma2_rn(make_float2(s[64 * H + c], s[64 * H + c + 1]), sl2, nm);
+        const bool poly = ((c >> 1) % kPolyPeriod) >= kPolyPeriod - kPolyPairs;
+        const float2 pp = poly ? exp2_poly2(xx) : make_float2(ex2_approx(xx.x), ex2_approx(xx.y));
+        a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], pp);
+        uint32_t pb;
+        if constexpr (kPackTruncate) {
+            pb = __byte_perm(__float_as_uint(pp.x), __float_as_uint(pp.y), 0x7632);
+            b2[(c >> 1) & 3] = __fadd2_rn(b2[(c >> 1) & 3], make_float2(__uint_as_float(pb << 16),
+                                                                        __uint_as_float(pb & 0xFFFF0000u)));
+        } else {
+            pb = pack_bf16x2(pp.x, pp.y);
+            b[(c >> 1) & 3] = add_bf16x2_to(b[(c >> 1) & 3], pb);
+        }
+        pk[c >> 1] = pb;
+    }
+    ls = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+    const float2 bb = __fadd2_rn(__fadd2_rn(b2[0], b2[1]), __fadd2_rn(b2[2], b2[3]));
+    lrs = ((b[0] + b[1]) + (b[2] + b[3])) + (bb.x + bb.y);
+}
+
+// ------------------------------------------------------------------ softmax
+// One warpgroup, query tile x; thread owns row (warp % 4) * 32 + lane.
+template <int D, bool O_BF16>
+__device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
+                                             uint32_t tmem, int x, int warp, int lane) {
+    using C = Cfg<D>;
+    const int row_in_tile = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float LN2 = 0.69314718055994530942f;
+    const float NEG_INF = __int_as_float(0xff800000);
+    uint64_t *s_full = &bars[C::kBarSFull + x];
+    uint64_t *p_full = &bars[C::kBarPFull + x];
+    uint64_t *o_final = &bars[C::kBarOFinal + x];
+    uint64_t *o_free = &bars[C::kBarOFree + x];
+    const uint32_t t_s = tmem + lane_off + col_s(x);
+    const uint32_t t_o = tmem + lane_off + col_o(x, D);
+    uint32_t gs = 0;  // S tiles of this query tile consumed so far (s_full / p_full phase)
+    uint32_t tl = 0;  // units in which this query tile had work (o_final / o_free phase)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+        const int t = unit_index(k);
+        if (t >= p.n_units) break;
+        const UnitCoord u = decode_unit(p, t);
+        const int row = u.blk * kUnitRows + x * BM + row_in_tile;
+        const bool row_valid = row < p.N;
+        const size_t row_id = (size_t)u.bh * p.N + row;
+        const int n = u.n[x];
+        if (n == 0) {  // no allowed key for these rows: O = 0, lse = -inf
+            if (row_valid) fill_row<D, O_BF16>(p.o, p.lse, row_id, false, NEG_INF);
+            continue;
+        }
+        int lim = p.N;
+        if (p.k_len) lim = min(max(__ldg(p.k_len + u.b), 0), p.N);
+        if (p.causal) lim = min(lim, row + 1);
+
+        float m_ref = 0.f;  // reference maximum, log2 units
+        float l = 0.f;      // running sum of 2^(x - m_ref), unrounded: gives lse
+        float lr = 0.f;     // running sum of bf16(2^(x - m_ref)), the weights the tensor core
+                            // multiplies V by: dividing O by it makes O an exact convex
+                            // combination of V rows (a lone dominant weight is not rounded away)
+        for (int j = 0; j < n; ++j, ++gs) {
+            ok = mbar_wait(s_full, gs & 1, abort_flag, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+
+            const int kv0 = j * BN;
+            const bool masked = kv0 + BN > lim;  // masking step: keys at or beyond the row's limit
+            float s[BN];
+            uint32_t pk0[32], pk1[32];          // P for keys [0,64) and [64,128), two bf16 per column
+            float2 ls = make_float2(0.f, 0.f);  // this tile's unrounded sum (packed pair)
+            float lrs = 0.f;                    // this tile's rounded (bf16) sum
+            if (j == 0) {
+                // first key tile of the unit: the row maximum comes first
+                load_scores<0>(t_s, s);
+                load_scores<1>(t_s, s);
+                if (masked) mask_scores<0>(s, kv0, lim);
+                if (masked) mask_scores<1>(s, kv0, lim);
+                const float m_new = fmaxf(max64(s), max64(s + 64)) * p.scale_log2;
+                m_ref = (m_new == NEG_INF) ? 0.f : m_new;
+                l = 0.f;
+                lr = 0.f;
+                exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
+                tmem_st32(t_s + 0, pk0);
+                exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
+            } else {
+                // Later tiles: the first half's exponentials are taken against
+                // the current reference while the second half is still in flight
+                // from TMEM; only if the row maximum exceeds the reference by more
+                // than tau is the first half recomputed (its scores reloaded from
+                // TMEM, untouched until P is stored) and O rescaled.
+                load_scores<0>(t_s, s);
+                tmem_ld32f(t_s + 64, s + 64);  // second half stays in flight
+                tmem_ld32f(t_s + 96, s + 96);
+                if (masked) mask_scores<0>(s, kv0, lim);
+                const float mx0 = max64(s);
+                exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
+                tmem_ld_wait();
+                tmem_reg_fence_f<64>(s + 64);
+                if (masked) mask_scores<1>(s, kv0, lim);
+                const float m_new = fmaxf(mx0, max64(s + 64)) * p.scale_log2;
+                float alpha = 1.f;
+                bool redo = false;
+                if (m_new > m_ref + p.tau) {
+                    alpha = ex2_approx(m_ref - m_new);
+                    m_ref = m_new;
+                    redo = true;
+                }
+                if (__any_sync(0xffffffffu, redo)) {
+                    // O_X holds P_X V for key tiles < j and nothing is adding to
+                    // it: the commit that released S_X(j) covered the last such
+                    // product, and the next one waits for this tile's P.
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        uint32_t r[32];
+                        tmem_ld32(t_o + ch * 32, r);
+                        tmem_ld_wait();
+                        tmem_reg_fence(r);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+                        tmem_st32(t_o + ch * 32, r);
+                    }
+                    l *= alpha;
+                    lr *= alpha;
+                    ls = make_float2(0.f, 0.f);
+                    lrs = 0.f;
+                    load_scores<0>(t_s, s);
+                    if (masked) mask_scores<0>(s, kv0, lim);
+                    exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
+                }
+                tmem_st32(t_s + 0, pk0);  // P overwrites S keys [0, 64), no longer needed
+                exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
+            }
+            tmem_st32(t_s + 32, pk1);
+            l += ls.x + ls.y;
+            lr += lrs;
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        if (ok) {
+            ok = mbar_wait(o_final, tl & 1, abort_flag, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (!ok) {  // abandon this unit: mark its rows
+            if (row_valid) fill_row<D, O_BF16>(p.o, p.lse, row_id, true, __int_as_float(0x7fc00000));
+            break;
+        }
+        tc_fence_after();
+        const float inv_l = 1.f / lr;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(t_o + ch * 32, r);
+            tmem_ld_wait();
+            tmem_reg_fence(r);
+            if (row_valid) store_row_chunk<D, O_BF16>(p.o, row_id, ch, r, inv_l);
+        }
+        if (row_valid) p.lse[row_id] = (m_ref + log2f(l)) * LN2;
+        tc_fence_before();
+        mbar_arrive(o_free);
+        ++tl;
+    }
+    return ok;
+}
+
+// ------------------------------------------------------------------ MMA issuer
+template <int D>
+__device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
+                                         uint32_t tmem, uint32_t q_addr, uint32_t k_addr, uint32_t v_addr) {
+    using C = Cfg<D>;
+    const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
+    const uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
+    // Descriptors differ only in their start-address field (bits [0,14), in
+    // 16-byte units), so each operand's descriptor is a base plus an offset.
+    const uint64_t q_desc = sw128_desc(q_addr, 16, 1024);
+    const uint64_t k_desc = sw128_desc(k_addr, 16, 1024);
+    const uint64_t v_desc = sw128_desc(v_addr, C::kChunkBytes, 1024);
+    uint32_t tq = 0;              // non-empty units (q_full phase)
+    uint32_t gk = 0, gv = 0;      // K and V ring positions
+    uint32_t gp0 = 0, gp1 = 0;    // P_X V products issued (p_full phase)
+    uint32_t tl0 = 0, tl1 = 0;    // units in which tile X had work (o_free phase)
+    const uint64_t to = p.timeout_ns;
+
+    // S_X = Q_X K^T for the key tile in ring slot kslot
+    auto qk = [&](int x, uint32_t kslot) {
+        const uint64_t qd = q_desc + ((x * C::kTileBytes) >> 4);
+        const uint64_t kd = k_desc + ((kslot * C::kTileBytes) >> 4);
+        if constexpr (D == 128) mma_ss_k128(tmem + col_s(x), qd, kd, idesc_qk, 0u);
+        else mma_ss_k64(tmem + col_s(x), qd, kd, idesc_qk, 0u);
+        tc_commit(&bars[C::kBarSFull + x]);
+    };
+    // O_X (+)= P_X V for the value tile in ring slot vslot; `first` starts a
+    // fresh accumulator, `last` ends the unit for tile X
+    auto pv = [&](int x, uint32_t &gpx, uint32_t tlx, uint32_t vslot, bool first, bool last) -> bool {
+        if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
+        ++gpx;
+        if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
+        tc_fence_after();
+        mma_ts_k128(tmem + col_o(x, D), tmem + col_s(x), v_desc + ((vslot * C::kTileBytes) >> 4), idesc_pv,
+                    first ? 0u : 1u);
+        if (last) tc_commit(&bars[C::kBarOFinal + x]);
+        return true;
+    };
+
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+        const int t = unit_index(k);
+        if (t >= p.n_units) break;
+        const UnitCoord u = decode_unit(p, t);
+        if (u.nmax == 0) continue;
+        if (!mbar_wait(&bars[C::kBarQFull], tq & 1, abort_flag, to)) { ok = false; break; }
+        ++tq;
+        tc_fence_after();
+        for (int j = 0; j <= u.nmax; ++j) {
+            // products with V_{j-1}, interleaved with the scores of key tile j
+            const bool have_k = j < u.nmax;
+            const uint32_t kslot = gk % C::kKStages, vslot = gv % C::kVStages;
+            if (have_k && !mbar_wait(&bars[C::kBarKFull + kslot], (gk / C::kKStages) & 1, abort_flag, to)) {
+                ok = false;
+                break;
+            }
+            if (j > 0 && !mbar_wait(&bars[C::kBarVFull + vslot], (gv / C::kVStages) & 1, abort_flag, to)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (j > 0 && j - 1 < u.n[0] && !pv(0, gp0, tl0, vslot, j == 1, j == u.n[0])) { ok = false; break; }
+            if (have_k && j < u.n[0]) qk(0, kslot);
+            if (j > 0 && j - 1 < u.n[1] && !pv(1, gp1, tl1, vslot, j == 1, j == u.n[1])) { ok = false; break; }
+            if (have_k && j < u.n[1]) qk(1, kslot);
+            if (j > 0) {
+                tc_commit(&bars[C::kBarVEmpty + vslot]);
+                ++gv;
+            }
+            if (have_k) {
+                tc_commit(&bars[C::kBarKEmpty + kslot]);
+                ++gk;
+                if (j == u.nmax - 1) tc_commit(&bars[C::kBarQEmpty]);
+            }
+        }
+        tl0 += u.n[0] > 0;
+        tl1 += u.n[1] > 0;
+    }
+    return ok;
+}
+
+// ------------------------------------------------------------------ TMA producer
+template <int D>
+__device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
+                                          uint8_t *sQ, uint8_t *sK, uint8_t *sV) {
+    using C = Cfg<D>;
+    prefetch_tensormap(&p.tm_q);
+    prefetch_tensormap(&p.tm_k);
+    prefetch_tensormap(&p.tm_v);
+    const uint64_t to = p.timeout_ns;
+    uint32_t tq = 0, gk = 0, gv = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+        const int t = unit_index(k);
+        if (t >= p.n_units) break;
+        const UnitCoord u = decode_unit(p, t);
+        if (u.nmax == 0) continue;
+        if (tq > 0 && !mbar_wait(&bars[C::kBarQEmpty], (tq - 1) & 1, abort_flag, to)) {
+            ok = false;
+            break;
+        }
+        mbar_arrive_expect_tx(&bars[C::kBarQFull], kQTiles * C::kTileBytes);
+#pragma unroll
+        for (int x = 0; x < kQTiles; ++x)
+#pragma unroll
+            for (int c = 0; c < C::kChunks; ++c)
+                tma_load_3d(sQ + x * C::kTileBytes + c * C::kChunkBytes, &p.tm_q, &bars[C::kBarQFull], c * 64,
+                            u.blk * kUnitRows + x * BM, u.bh);
+        ++tq;
+        for (int j = 0; j < u.nmax && ok; ++j) {
+            {
+                const uint32_t slot = gk % C::kKStages, round = gk / C::kKStages;
+                if (round > 0 && !mbar_wait(&bars[C::kBarKEmpty + slot], (round - 1) & 1, abort_flag, to)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&bars[C::kBarKFull + slot], C::kTileBytes);
+#pragma unroll
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(sK + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_k, &bars[C::kBarKFull + slot],
+                                c * 64, j * BN, u.bh);
+                ++gk;
+            }
+            {
+                const uint32_t slot = gv % C::kVStages, round = gv / C::kVStages;
+                if (round > 0 && !mbar_wait(&bars[C::kBarVEmpty + slot], (round - 1) & 1, abort_flag, to)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&bars[C::kBarVFull + slot], C::kTileBytes);
+#pragma unroll
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(sV + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_v, &bars[C::kBarVFull + slot],
+                                c * 64, j * BN, u.bh);
+                ++gv;
+            }
+        }
+    }
+    if (!ok) record_timeout(p);
+    // drain: every copy this thread issued has landed before the CTA may exit
+    if (tq > 0) mbar_wait_drain(&bars[C::kBarQFull], (tq - 1) & 1, to);
+    const uint32_t nk = gk < (uint32_t)C::kKStages ? gk : (uint32_t)C::kKStages;
+    for (uint32_t i = 0; i < nk; ++i) {
+        const uint32_t g = gk - 1 - i;
+        mbar_wait_drain(&bars[C::kBarKFull + g % C::kKStages], (g / C::kKStages) & 1, to);
+    }
+    const uint32_t nv = gv < (uint32_t)C::kVStages ? gv : (uint32_t)C::kVStages;
+    for (uint32_t i = 0; i < nv; ++i) {
+        const uint32_t g = gv - 1 - i;
+        mbar_wait_drain(&bars[C::kBarVFull + g % C::kVStages], (g / C::kVStages) & 1, to);
+    }
 }
 
 template <int D, bool O_BF16>
@@ -152,9 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
-            uint32_t cnt = 1;
-            if (i == C::kBarPFull || i == C::kBarPFull + 1 || i == C::kBarOFree) cnt = kSoftmaxWarps * 32;
-            mbar_init(&bars[i], cnt);
+            const bool per_row =
+                (i >= C::kBarPFull && i < C::kBarPFull + 2) || (i >= C::kBarOFree && i < C::kBarOFree + 2);
+            mbar_init(&bars[i], per_row ? 128u : 1u);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -169,322 +609,20 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
     const uint32_t tmem = *tmem_slot;
 
     if (warp < kSoftmaxWarps) {
-        // ------------------------------------------------------------ softmax
-        const int row_in_tile = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const float LN2 = 0.69314718055994530942f;
-        const float NEG_INF = __int_as_float(0xff800000);
-        uint32_t g = 0;   // global key-tile counter (same sequence as the MMA issuer)
-        uint32_t tl = 0;  // non-empty work units seen
-        bool ok = true;
-        for (int k = 0; ok; ++k) {
-            const int t = unit_index(k);
-            if (t >= p.n_tiles) break;
-            const TileCoord tc = decode_tile(p, t);
-            const int row = tc.qt * BM + row_in_tile;
-            const bool row_valid = row < p.N;
-            const size_t row_id = (size_t)tc.bh * p.N + row;
-            int lim = p.N;
-            if (p.k_len) lim = min(max(__ldg(p.k_len + tc.b), 0), p.N);
-            if (p.causal) lim = min(lim, row + 1);
-
-            if (tc.n_kv == 0) {  // no allowed key in this unit: O = 0, lse = -inf
-                if (row_valid) {
-                    if constexpr (O_BF16) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + row_id * D);
-                        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-                    } else {
-                        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.o) + row_id * D);
-                        for (int i = 0; i < D / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                    p.lse[row_id] = NEG_INF;
-                }
-                continue;
-            }
-
-            float m_ref = 0.f;  // reference maximum, log2 units
-            float l = 0.f;      // running sum of 2^(x - m_ref), unrounded: gives lse
-            float lr = 0.f;     // running sum of bf16(2^(x - m_ref)), the weights the tensor core
-                                // multiplies V by: dividing O by it makes O an exact convex
-                                // combination of V rows (a lone dominant weight is not rounded away)
-            for (int j = 0; j < tc.n_kv; ++j, ++g) {
-                const uint32_t buf = g & 1;
-                ok = mbar_wait(&bars[C::kBarSFull + buf], (g >> 1) & 1, abort_flag, p.timeout_ns);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                tc_fence_after();
-
-                float s[BN];
-                {
-                    uint32_t r0[32], r1[32], r2[32], r3[32];
-                    const uint32_t a = tmem + lane_off + col_s(buf);
-                    tmem_ld32(a + 0, r0);
-                    tmem_ld32(a + 32, r1);
-                    tmem_ld32(a + 64, r2);
-                    tmem_ld32(a + 96, r3);
-                    tmem_ld_wait();
-                    tmem_reg_fence(r0);
-                    tmem_reg_fence(r1);
-                    tmem_reg_fence(r2);
-                    tmem_reg_fence(r3);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        s[c] = __uint_as_float(r0[c]);
-                        s[32 + c] = __uint_as_float(r1[c]);
-                        s[64 + c] = __uint_as_float(r2[c]);
-                        s[96 + c] = __uint_as_float(r3[c]);
-                    }
-                }
-                const int kv0 = j * BN;
-                if (kv0 + BN > lim) {  // masking step: keys at or beyond the row's limit
-#pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if (kv0 + c >= lim) s[c] = NEG_INF;
-                }
-                float mx[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = s[i];
-#pragma unroll
-                for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-                const float rowmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                const float m_new = rowmax * p.scale_log2;
-                float alpha = 1.f;
-                bool resc = false;
-                if (j == 0) {
-                    m_ref = (m_new == NEG_INF) ? 0.f : m_new;
-                    l = 0.f;
-                    lr = 0.f;
-                } else if (m_new > m_ref + p.tau) {
-                    alpha = ex2_approx(m_ref - m_new);
-                    l *= alpha;
-                    lr *= alpha;
-                    m_ref = m_new;
-                    resc = true;
-                }
-                const float neg_m = -m_ref;
-                float ls[8], lrs[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) ls[i] = lrs[i] = 0.f;
-                uint32_t pk0[32], pk1[32];  // keys [0,64) and [64,128), two bf16 per column
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, neg_m));
-                    const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, neg_m));
-                    ls[(c >> 1) & 7] += p0 + p1;
-                    pk0[c >> 1] = pack_bf16x2(p0, p1);
-                    lrs[(c >> 1) & 7] += bf16x2_lo(pk0[c >> 1]) + bf16x2_hi(pk0[c >> 1]);
-                }
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const float p0 = ex2_approx(fmaf(s[64 + c], p.scale_log2, neg_m));
-                    const float p1 = ex2_approx(fmaf(s[64 + c + 1], p.scale_log2, neg_m));
-                    ls[(c >> 1) & 7] += p0 + p1;
-                    pk1[c >> 1] = pack_bf16x2(p0, p1);
-                    lrs[(c >> 1) & 7] += bf16x2_lo(pk1[c >> 1]) + bf16x2_hi(pk1[c >> 1]);
-                }
-                l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-                lr += ((lrs[0] + lrs[1]) + (lrs[2] + lrs[3])) + ((lrs[4] + lrs[5]) + (lrs[6] + lrs[7]));
-                {
-                    const uint32_t a = tmem + lane_off + col_p(buf);
-                    tmem_st32(a + 0, pk0);
-                    tmem_st32(a + 32, pk1);
-                }
-                if (__any_sync(0xffffffffu, resc)) {
-                    // O holds P_0..P_{g-1} V; wait for the last of those products,
-                    // then scale this warp's 32 rows in place.
-                    ok = mbar_wait(&bars[C::kBarODone], (g - 1) & 1, abort_flag, p.timeout_ns);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int ch = 0; ch < D / 32; ++ch) {
-                        uint32_t r[32];
-                        const uint32_t a = tmem + lane_off + kColO + ch * 32;
-                        tmem_ld32(a, r);
-                        tmem_ld_wait();
-                        tmem_reg_fence(r);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-                        tmem_st32(a, r);
-                    }
-                }
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&bars[C::kBarPFull + buf]);
-            }
-            if (ok) {
-                ok = mbar_wait(&bars[C::kBarOFinal], tl & 1, abort_flag, p.timeout_ns);
-                ok = __all_sync(0xffffffffu, ok);
-            }
-            if (!ok) {
-                // abandon this unit: mark its rows
-                if (row_valid) {
-                    const float nan = __int_as_float(0x7fc00000);
-                    if constexpr (O_BF16) {
-                        uint16_t *dst = reinterpret_cast<uint16_t *>(p.o) + row_id * D;
-                        for (int i = 0; i < D; ++i) dst[i] = 0x7fc0;
-                    } else {
-                        float *dst = reinterpret_cast<float *>(p.o) + row_id * D;
-                        for (int i = 0; i < D; ++i) dst[i] = nan;
-                    }
-                    p.lse[row_id] = nan;
-                }
-                break;
-            }
-            tc_fence_after();
-            const float inv_l = 1.f / lr;
-#pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_off + kColO + ch * 32, r);
-                tmem_ld_wait();
-                tmem_reg_fence(r);
-                if (row_valid) {
-                    if constexpr (O_BF16) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.o) + row_id * D + ch * 32);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l);
-                            v.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l);
-                            v.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l);
-                            v.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l);
-                            dst[i] = v;
-                        }
-                    } else {
-                        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.o) + row_id * D + ch * 32);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = make_float4(__uint_as_float(r[4 * i + 0]) * inv_l, __uint_as_float(r[4 * i + 1]) * inv_l,
-                                                 __uint_as_float(r[4 * i + 2]) * inv_l, __uint_as_float(r[4 * i + 3]) * inv_l);
-                    }
-                }
-            }
-            if (row_valid) p.lse[row_id] = (m_ref + log2f(l)) * LN2;
-            tc_fence_before();
-            mbar_arrive(&bars[C::kBarOFree]);
-            ++tl;
-        }
-        if (!ok) record_timeout(p);
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer
+        setmaxnreg_inc<kSoftmaxRegs>();
+        if (!softmax_role<D, O_BF16>(p, bars, abort_flag, tmem, warp >> 2, warp, lane)) record_timeout(p);
+    } else {
+        setmaxnreg_dec<kControlRegs>();
+    }
+    if (warp == kMmaWarp) {
         if (lane == 0) {
-            const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-            const uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
-            const uint32_t q_addr = smem_u32(sQ);
-            const uint32_t k_addr = smem_u32(sK);
-            const uint32_t v_addr = smem_u32(sV);
-            uint32_t g = 0, tl = 0;
-            bool ok = true;
-            // the one P V product whose issue is deferred behind the next Q K^T
-            bool pend = false;
-            uint32_t pend_g = 0, pend_tl = 0;
-            bool pend_first = false, pend_last = false;
-
-            auto issue_pv = [&](uint32_t pg, uint32_t ptl, bool first, bool last) -> bool {
-                const uint32_t stage = pg % C::kStages, round = pg / C::kStages, buf = pg & 1;
-                if (!mbar_wait(&bars[C::kBarVFull + stage], round & 1, abort_flag, p.timeout_ns)) return false;
-                if (!mbar_wait(&bars[C::kBarPFull + buf], (pg >> 1) & 1, abort_flag, p.timeout_ns)) return false;
-                if (first && ptl > 0) {  // previous unit's epilogue must have read O
-                    if (!mbar_wait(&bars[C::kBarOFree], (ptl - 1) & 1, abort_flag, p.timeout_ns)) return false;
-                }
-                tc_fence_after();
-                const uint32_t vs = v_addr + stage * C::kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bdesc = sw128_desc(vs + kk * 16 * 128, C::kChunkBytes, 1024);
-                    mma_ts(tmem + kColO, tmem + col_p(buf) + kk * 8, bdesc, idesc_pv, (first && kk == 0) ? 0u : 1u);
-                }
-                tc_commit(&bars[C::kBarKVEmpty + stage]);
-                tc_commit(&bars[C::kBarODone]);
-                if (last) tc_commit(&bars[C::kBarOFinal]);
-                return true;
-            };
-
-            for (int k = 0; ok; ++k) {
-                const int t = unit_index(k);
-                if (t >= p.n_tiles) break;
-                const TileCoord tc = decode_tile(p, t);
-                if (tc.n_kv == 0) continue;
-                if (!mbar_wait(&bars[C::kBarQFull], tl & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
-                tc_fence_after();
-                for (int j = 0; j < tc.n_kv; ++j, ++g) {
-                    const uint32_t stage = g % C::kStages, round = g / C::kStages, buf = g & 1;
-                    if (!mbar_wait(&bars[C::kBarKFull + stage], round & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t ks = k_addr + stage * C::kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                        mma_ss(tmem + col_s(buf), sw128_desc(q_addr + off, 16, 1024), sw128_desc(ks + off, 16, 1024),
-                               idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    tc_commit(&bars[C::kBarSFull + buf]);
-                    if (j == tc.n_kv - 1) tc_commit(&bars[C::kBarQEmpty]);
-                    if (pend && !issue_pv(pend_g, pend_tl, pend_first, pend_last)) { ok = false; break; }
-                    pend = true;
-                    pend_g = g;
-                    pend_tl = tl;
-                    pend_first = (j == 0);
-                    pend_last = (j == tc.n_kv - 1);
-                }
-                ++tl;
-            }
-            if (ok && pend) ok = issue_pv(pend_g, pend_tl, pend_first, pend_last);
-            if (!ok) record_timeout(p);
+            if (!mma_role<D>(p, bars, abort_flag, tmem, smem_u32(sQ), smem_u32(sK), smem_u32(sV))) record_timeout(p);
             // drain: no MMA may still be running when TMEM is released
             tc_commit(&bars[C::kBarDrain]);
             mbar_wait_drain(&bars[C::kBarDrain], 0, p.timeout_ns);
         }
     } else if (warp == kLoadWarp) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            prefetch_tensormap(&p.tm_q);
-            prefetch_tensormap(&p.tm_k);
-            prefetch_tensormap(&p.tm_v);
-            uint32_t g = 0, tl = 0;
-            bool ok = true;
-            for (int k = 0; ok; ++k) {
-                const int t = unit_index(k);
-                if (t >= p.n_tiles) break;
-                const TileCoord tc = decode_tile(p, t);
-                if (tc.n_kv == 0) continue;
-                if (tl > 0 && !mbar_wait(&bars[C::kBarQEmpty], (tl - 1) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
-                mbar_arrive_expect_tx(&bars[C::kBarQFull], C::kTileBytes);
-#pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(sQ + c * C::kChunkBytes, &p.tm_q, &bars[C::kBarQFull], c * 64, tc.qt * BM, tc.bh);
-                ++tl;
-                for (int j = 0; j < tc.n_kv; ++j, ++g) {
-                    const uint32_t stage = g % C::kStages, round = g / C::kStages;
-                    if (round > 0 && !mbar_wait(&bars[C::kBarKVEmpty + stage], (round - 1) & 1, abort_flag, p.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *ks = sK + stage * C::kTileBytes;
-                    uint8_t *vs = sV + stage * C::kTileBytes;
-                    mbar_arrive_expect_tx(&bars[C::kBarKFull + stage], C::kTileBytes);
-#pragma unroll
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_3d(ks + c * C::kChunkBytes, &p.tm_k, &bars[C::kBarKFull + stage], c * 64, j * BN, tc.bh);
-                    mbar_arrive_expect_tx(&bars[C::kBarVFull + stage], C::kTileBytes);
-#pragma unroll
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_3d(vs + c * C::kChunkBytes, &p.tm_v, &bars[C::kBarVFull + stage], c * 64, j * BN, tc.bh);
-                }
-            }
-            if (!ok) record_timeout(p);
-            // drain: every copy this thread issued has landed before the CTA may exit
-            if (tl > 0) mbar_wait_drain(&bars[C::kBarQFull], (tl - 1) & 1, p.timeout_ns);
-            const uint32_t n_last = g < (uint32_t)C::kStages ? g : (uint32_t)C::kStages;
-            for (uint32_t i = 0; i < n_last; ++i) {
-                const uint32_t gg = g - 1 - i;
-                const uint32_t stage = gg % C::kStages, round = gg / C::kStages;
-                mbar_wait_drain(&bars[C::kBarKFull + stage], round & 1, p.timeout_ns);
-                mbar_wait_drain(&bars[C::kBarVFull + stage], round & 1, p.timeout_ns);
-            }
-        }
+        if (lane == 0) load_role<D>(p, bars, abort_flag, sQ, sK, sV);
     }
 
     tc_fence_before();

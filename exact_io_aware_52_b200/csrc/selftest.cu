@@ -5,7 +5,7 @@
 //   * O = P V with tcgen05.mma, P packed into TMEM by tcgen05.st, V MN-major
 //     in shared memory;
 //   * the bounded mbarrier wait running out on a barrier nobody arrives at.
-// They use exactly the descriptor builders and wrappers of the kernel.
+// They use exactly the descriptor builders and MMA issue blocks of the kernel.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -91,11 +91,9 @@ __global__ void k_mma_ss(const __grid_constant__ SelfParams sp) {
         if (ok) {
             tc_fence_after();
             const uint32_t idesc = idesc_bf16_f32(128, 128, false);
-            for (int kk = 0; kk < sp.K / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_ss(tmem, sw128_desc(smem_u32(sA) + off, 16, 1024), sw128_desc(smem_u32(sB) + off, 16, 1024),
-                       idesc, kk > 0);
-            }
+            const uint64_t da = sw128_desc(smem_u32(sA), 16, 1024), db = sw128_desc(smem_u32(sB), 16, 1024);
+            if (sp.K == 128) mma_ss_k128(tmem, da, db, idesc, 0u);
+            else mma_ss_k64(tmem, da, db, idesc, 0u);
         }
         tc_commit(&bars[1]);
     }
@@ -175,9 +173,7 @@ __global__ void k_mma_ts(const __grid_constant__ SelfParams sp) {
         if (ok) {
             tc_fence_after();
             const uint32_t idesc = idesc_bf16_f32(128, D, true);
-            for (int kk = 0; kk < 8; ++kk)
-                mma_ts(tmem + colO, tmem + colP + kk * 8, sw128_desc(smem_u32(sV) + kk * 2048, 16384, 1024), idesc,
-                       kk > 0);
+            mma_ts_k128(tmem + colO, tmem + colP, sw128_desc(smem_u32(sV), 16384, 1024), idesc, 0u);
         }
         tc_commit(&bars[1]);
     }
@@ -218,6 +214,15 @@ __global__ void k_wait_timeout(int32_t *status, uint64_t timeout_ns) {
     __syncthreads();
     const bool ok = mbar_wait(&bar, 0, &abort_flag, timeout_ns);
     if (!ok) set_status(status, 5);
+}
+
+// y[i] = 2^x[i] through the FMA-pipe polynomial (pairs of lanes), n even.
+__global__ void k_exp2_poly(const float *x, float *y, int n) {
+    for (int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 2 * gridDim.x * blockDim.x) {
+        const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+        y[i] = r.x;
+        y[i + 1] = r.y;
+    }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
@@ -291,6 +296,13 @@ int fa_selftest_mma_ts(const void *p, const void *v, float *o, int D, int32_t *s
     const int smem = 32768 + 128 + 1024;
     if (cudaFuncSetAttribute(k_mma_ts, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 4;
     k_mma_ts<<<1, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(sp);
+    return finish(stream);
+}
+
+int fa_selftest_exp2_poly(const float *x, float *y, int n, void *stream) {
+    if (n < 0 || (n & 1)) return 1;
+    if (n == 0) return 0;
+    k_exp2_poly<<<64, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
     return finish(stream);
 }
 

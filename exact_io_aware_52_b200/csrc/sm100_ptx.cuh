@@ -71,6 +71,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// ---------------------------------------------------------------- registers
+// Per-warpgroup register reallocation; executed by all 128 threads of a
+// warpgroup.  The increases of some warpgroups must be covered by the
+// decreases of others within the registers the block was launched with.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- TMA
 // 3-D tiled bulk tensor load global -> shared, completion signalled on `bar`
 // as transaction bytes.  `map` is the generic address of a __grid_constant__
@@ -135,6 +148,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+// As tmem_ld32, into 32 consecutive floats.
+__device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float *f) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3]), "=f"(f[4]), "=f"(f[5]), "=f"(f[6]), "=f"(f[7]),
+          "=f"(f[8]), "=f"(f[9]), "=f"(f[10]), "=f"(f[11]), "=f"(f[12]), "=f"(f[13]), "=f"(f[14]),
+          "=f"(f[15]), "=f"(f[16]), "=f"(f[17]), "=f"(f[18]), "=f"(f[19]), "=f"(f[20]), "=f"(f[21]),
+          "=f"(f[22]), "=f"(f[23]), "=f"(f[24]), "=f"(f[25]), "=f"(f[26]), "=f"(f[27]), "=f"(f[28]),
+          "=f"(f[29]), "=f"(f[30]), "=f"(f[31])
+        : "r"(taddr));
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_reg_fence_f(float *f) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(f[i])::"memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 template <int N>
@@ -152,6 +185,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
         "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
         "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
 
@@ -209,11 +251,98 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
+// A whole K loop of tcgen05.mma issued back to back from one asm block, the
+// per-step descriptors formed in-line (base + start-address offset in 16-byte
+// units) so the issuing thread needs no registers for them.
+//
+// S (+)= A B^T over K = 16 * steps with both operands K-major, 128-byte
+// swizzled, stored as 64-element column blocks of `block_bytes` each: step kk
+// starts (kk / 4) * block_bytes + (kk % 4) * 32 bytes into both A and B.
+// The first step overwrites D when `accumulate` is 0.
+#define FA_SS_STEP(OFF)                                      \
+    "add.s64 da, %1, " #OFF ";\n\t"                          \
+    "add.s64 db, %2, " #OFF ";\n\t"                          \
+    "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, pt;\n\t"
+__device__ __forceinline__ void mma_ss_k64(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    // K = 64: one column block, offsets 0, 32, 64, 96 bytes
+    asm volatile(
+        "{\n\t.reg .b64 da, db;\n\t.reg .pred p, pt;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 pt, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        FA_SS_STEP(2) FA_SS_STEP(4) FA_SS_STEP(6)
+        "}" ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ss_k128(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    // K = 128: two column blocks of 16384 bytes (1024 in 16-byte units)
+    asm volatile(
+        "{\n\t.reg .b64 da, db;\n\t.reg .pred p, pt;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 pt, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        FA_SS_STEP(2) FA_SS_STEP(4) FA_SS_STEP(6)
+        FA_SS_STEP(1024) FA_SS_STEP(1026) FA_SS_STEP(1028) FA_SS_STEP(1030)
+        "}" ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+#undef FA_SS_STEP
+
+// O (+)= P V over 128 keys (8 steps of K = 16): P in TMEM from column a_tmem
+// (8 columns per step), V MN-major in shared memory, 16 key rows of 128 bytes
+// per step (2048 bytes = 128 in 16-byte units).
+#define FA_TS_STEP(TA, DB)                                   \
+    "add.u32 ta, %1, " #TA ";\n\t"                           \
+    "add.s64 db, %2, " #DB ";\n\t"                           \
+    "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, pt;\n\t"
+__device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t.reg .pred p, pt;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 pt, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        FA_TS_STEP(8, 128) FA_TS_STEP(16, 256) FA_TS_STEP(24, 384) FA_TS_STEP(32, 512)
+        FA_TS_STEP(40, 640) FA_TS_STEP(48, 768) FA_TS_STEP(56, 896)
+        "}" ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+#undef FA_TS_STEP
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x for two lanes on the FMA pipe (the MUFU ex2 unit is the other source of
+// exponentials; splitting the work between the two pipes keeps either from
+// capping the tile rate).  Cody-Waite style reduction x = n + f with
+// n = round(x) taken from the low mantissa bits of x + 1.5*2^23 and
+// f in [-1/2, 1/2]; 2^f by a degree-4 polynomial with p(0) = 1 whose
+// coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
+// exchange, fitted for this file; max relative error 3.6e-6 evaluated in
+// fp32); 2^n enters by adding n to the exponent field.  Inputs below -127
+// are clamped there, giving +0 up to the polynomial's error; inputs must be
+// below 128.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -127.f);
+    x.y = fmaxf(x.y, -127.f);
+    const float2 t = __fadd2_rn(x, magic);  // round(x) + magic, exact integer arithmetic
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));  // exact: |f| <= 1/2
+    float2 q = __ffma2_rn(make_float2(0.009782912209630013f, 0.009782912209630013f), f,
+                          make_float2(0.055976882576942444f, 0.055976882576942444f));
+    q = __ffma2_rn(q, f, make_float2(0.24020710587501526f, 0.24020710587501526f));
+    q = __ffma2_rn(q, f, make_float2(0.6931136250495911f, 0.6931136250495911f));
+    q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+    // low bits of t hold n (two's complement within the mantissa): bits(t) << 23 == n << 23
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // Packs two floats as bf16 (round to nearest even): `lo` in bits [0,16),
@@ -222,6 +351,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// acc + lo(u) + hi(u), each bf16 half of the packed pair widened exactly and
+// added in fp32 (mixed-precision add, one instruction per half).
+__device__ __forceinline__ float add_bf16x2_to(float acc, uint32_t u) {
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %1;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\t"
+        "add.rn.f32.bf16 %0, hi, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(u));
+    return acc;
 }
 
 // The two bf16 halves of a packed pair, widened exactly to float.

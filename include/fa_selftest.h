@@ -40,6 +40,11 @@ FA_SELFTEST_EXPORT int fa_selftest_mma_ss(const void *a, const void *b, float *s
 FA_SELFTEST_EXPORT int fa_selftest_mma_ts(const void *p, const void *v, float *o, int D, int32_t *status,
                                           void *stream);
 
+/* y[i] = 2^x[i] (fp32, n even) through the FMA-pipe polynomial exponential the
+ * kernel uses for part of its softmax weights (the online softmax of section
+ * "Calculo de Softmax en linea"); inputs below -127 give +0. */
+FA_SELFTEST_EXPORT int fa_selftest_exp2_poly(const float *x, float *y, int n, void *stream);
+
 /* Wait on a barrier nothing arrives at, with a limit of timeout_ms; the wait
  * must give up and store 5 in *status. */
 FA_SELFTEST_EXPORT int fa_selftest_wait_timeout(int32_t *status, uint32_t timeout_ms, void *stream);

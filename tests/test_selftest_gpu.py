@@ -88,3 +88,25 @@ def test_bounded_wait_gives_up():
     assert dt < 5.0
     x = torch.ones(16, device=_dev())
     assert float((x * 2).sum().item()) == 32.0
+
+
+def test_polynomial_exp2_error_bound():
+    """The FMA-pipe 2^x: relative error <= 4e-6 against float64 exp2 over the
+    range the softmax feeds it ([-127, 8]), exact powers of two at integers
+    (p(0) = 1), and +0 (to within the error) for inputs at or below -127."""
+    lib = fb.load_selftest()
+    x = torch.cat([torch.linspace(-126.0, 8.0, 1 << 20), torch.arange(-126, 9, dtype=torch.float32),
+                   torch.tensor([-127.0, -200.0, -1e30, float("-inf")])])
+    if x.numel() % 2:
+        x = torch.cat([x, torch.zeros(1)])
+    xd = x.to(_dev())
+    y = torch.empty_like(xd)
+    assert lib.fa_selftest_exp2_poly(_p(xd), _p(y), x.numel(), None) == 0
+    yy = y.cpu().double()
+    ref = torch.exp2(x.double())
+    live = x >= -126
+    rel = ((yy[live] - ref[live]) / ref[live]).abs()
+    assert rel.max().item() <= 4e-6, rel.max().item()
+    ints = (x == x.round()) & live
+    assert torch.equal(yy[ints], ref[ints])
+    assert (yy[~live].abs() <= 1e-43).all()

@@ -223,15 +223,6 @@ __device__ __forceinline__ float max64(const float *v) {
     return fmaxf(fmax3(a0, a1, a2), a3);
 }
 
-// Scores of keys [64H, 64H+64) of this thread's row: two 32-column TMEM loads.
-template <int H>
-__device__ __forceinline__ void load_scores(uint32_t t_s, float *s) {
-    tmem_ld32f(t_s + 64 * H, s + 64 * H);
-    tmem_ld32f(t_s + 64 * H + 32, s + 64 * H + 32);
-    tmem_ld_wait();
-    tmem_reg_fence_f<64>(s + 64 * H);
-}
-
 // Masking step for keys [64H, 64H+64) of a tile starting at key kv0: keys at
 // or beyond the row's limit get -inf.
 template <int H>
@@ -327,67 +318,49 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             uint32_t pk0[32], pk1[32];          // P for keys [0,64) and [64,128), two bf16 per column
             float2 ls = make_float2(0.f, 0.f);  // this tile's unrounded sum (packed pair)
             float lrs = 0.f;                    // this tile's rounded (bf16) sum
+            // the row's 128 scores: four 32-column TMEM loads, one wait
+            tmem_ld32f(t_s + 0, s);
+            tmem_ld32f(t_s + 32, s + 32);
+            tmem_ld32f(t_s + 64, s + 64);
+            tmem_ld32f(t_s + 96, s + 96);
+            tmem_ld_wait();
+            tmem_reg_fence_f<BN>(s);
+            if (masked) {
+                mask_scores<0>(s, kv0, lim);
+                mask_scores<1>(s, kv0, lim);
+            }
+            const float m_new = fmaxf(max64(s), max64(s + 64)) * p.scale_log2;
+            float alpha = 1.f;
+            bool resc = false;
             if (j == 0) {
-                // first key tile of the unit: the row maximum comes first
-                load_scores<0>(t_s, s);
-                load_scores<1>(t_s, s);
-                if (masked) mask_scores<0>(s, kv0, lim);
-                if (masked) mask_scores<1>(s, kv0, lim);
-                const float m_new = fmaxf(max64(s), max64(s + 64)) * p.scale_log2;
                 m_ref = (m_new == NEG_INF) ? 0.f : m_new;
                 l = 0.f;
                 lr = 0.f;
-                exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
-                tmem_st32(t_s + 0, pk0);
-                exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
-            } else {
-                // Later tiles: the first half's exponentials are taken against
-                // the current reference while the second half is still in flight
-                // from TMEM; only if the row maximum exceeds the reference by more
-                // than tau is the first half recomputed (its scores reloaded from
-                // TMEM, untouched until P is stored) and O rescaled.
-                load_scores<0>(t_s, s);
-                tmem_ld32f(t_s + 64, s + 64);  // second half stays in flight
-                tmem_ld32f(t_s + 96, s + 96);
-                if (masked) mask_scores<0>(s, kv0, lim);
-                const float mx0 = max64(s);
-                exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
-                tmem_ld_wait();
-                tmem_reg_fence_f<64>(s + 64);
-                if (masked) mask_scores<1>(s, kv0, lim);
-                const float m_new = fmaxf(mx0, max64(s + 64)) * p.scale_log2;
-                float alpha = 1.f;
-                bool redo = false;
-                if (m_new > m_ref + p.tau) {
-                    alpha = ex2_approx(m_ref - m_new);
-                    m_ref = m_new;
-                    redo = true;
-                }
-                if (__any_sync(0xffffffffu, redo)) {
-                    // O_X holds P_X V for key tiles < j and nothing is adding to
-                    // it: the commit that released S_X(j) covered the last such
-                    // product, and the next one waits for this tile's P.
-#pragma unroll
-                    for (int ch = 0; ch < D / 32; ++ch) {
-                        uint32_t r[32];
-                        tmem_ld32(t_o + ch * 32, r);
-                        tmem_ld_wait();
-                        tmem_reg_fence(r);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-                        tmem_st32(t_o + ch * 32, r);
-                    }
-                    l *= alpha;
-                    lr *= alpha;
-                    ls = make_float2(0.f, 0.f);
-                    lrs = 0.f;
-                    load_scores<0>(t_s, s);
-                    if (masked) mask_scores<0>(s, kv0, lim);
-                    exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
-                }
-                tmem_st32(t_s + 0, pk0);  // P overwrites S keys [0, 64), no longer needed
-                exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
+            } else if (m_new > m_ref + p.tau) {
+                alpha = ex2_approx(m_ref - m_new);
+                l *= alpha;
+                lr *= alpha;
+                m_ref = m_new;
+                resc = true;
             }
+            if (__any_sync(0xffffffffu, resc)) {
+                // O_X holds P_X V for key tiles < j and nothing is adding to it:
+                // the commit that released S_X(j) covered the last such product,
+                // and the next one waits for this tile's P.  Scale in place.
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t r[32];
+                    tmem_ld32(t_o + ch * 32, r);
+                    tmem_ld_wait();
+                    tmem_reg_fence(r);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+                    tmem_st32(t_o + ch * 32, r);
+                }
+            }
+            exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
+            tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
+            exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
             tmem_st32(t_s + 32, pk1);
             l += ls.x + ls.y;
             lr += lrs;

@@ -143,11 +143,12 @@ __device__ __forceinline__ int unit_index(int k) {
     return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
+// Units are numbered head-major (the CTAs working at one time share a few
+// heads' K and V in L2), longest (causal) query blocks first within a head.
 __device__ __forceinline__ UnitCoord decode_unit(const FwdParams &p, int t) {
     UnitCoord u;
-    const int BH = p.B * p.H;
-    u.blk = p.n_blocks - 1 - t / BH;  // longest (causal) query blocks first
-    u.bh = t % BH;
+    u.blk = p.n_blocks - 1 - t % p.n_blocks;
+    u.bh = t / p.n_blocks;
     u.b = u.bh / p.H;
     int kv_lim = p.N;
     if (p.k_len) kv_lim = min(max(__ldg(p.k_len + u.b), 0), p.N);

@@ -99,7 +99,7 @@ def algorithmic_bytes(w, k_len) -> float:
     """Compulsory HBM bytes of one launch: Q, K, V read once (valid keys only
     under key padding), O (fp32) and lse written once."""
     n_elem = w.B * w.H * w.N * w.d
-    kv_rows = w.H * (sum(min(max(int(x), 0), w.N) for x in k_len) if k_len is not None else w.B * w.N)
+    kv_rows = w.kv_heads * (sum(min(max(int(x), 0), w.N) for x in k_len) if k_len is not None else w.B * w.N)
     return 2.0 * n_elem + 2 * 2.0 * kv_rows * w.d + 4.0 * n_elem + 4.0 * w.B * w.H * w.N
 
 
@@ -356,7 +356,7 @@ def run_ours(args, world, rank, local):
         e1.record(stream)
         e1.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-        h2d = 3 * qh.numel() * 2 + (0 if klh is None else klh.numel() * 4)
+        h2d = (qh.numel() + kh.numel() + vh.numel()) * 2 + (0 if klh is None else klh.numel() * 4)
         d2h = oh.numel() * 4 + lh.numel() * 4
         e2e = {"value": flops * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
@@ -382,9 +382,10 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-                   "out": "fp32 O + fp32 lse", "flops_per_step_per_gpu": flops,
-                   "l2": "inputs larger than L2 (Q,K,V %.0f MB > 126 MB); no flush" % (3 * q.numel() * 2 / 1e6),
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "N": w.N, "d": w.d,
+                   "causal": w.causal, "out": "fp32 O + fp32 lse", "flops_per_step_per_gpu": flops,
+                   "l2": "inputs larger than L2 (Q,K,V %.0f MB > 126 MB); no flush"
+                         % ((q.numel() + k.numel() + v.numel()) * 2 / 1e6),
                    "parallelism": f"replicas x{world}"},
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": roofline,

@@ -38,7 +38,7 @@ class FaParams(ctypes.Structure):
         ("dev_status", ctypes.c_void_p),
         ("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int),
         ("causal", ctypes.c_int), ("scale", ctypes.c_float), ("o_dtype", ctypes.c_int),
-        ("flags", ctypes.c_int), ("timeout_ms", ctypes.c_uint32),
+        ("flags", ctypes.c_int), ("timeout_ms", ctypes.c_uint32), ("H_kv", ctypes.c_int),
     ]
 
 
@@ -148,15 +148,18 @@ def make_params(q, k, v, o, lse, causal, scale, k_len=None, dev_status=None, fla
         shape = tuple(q.shape)
     B, H, N, d = shape
     o_dtype = FA_O_BF16 if (o is not None and o.dtype == torch.bfloat16) else FA_O_F32
+    H_kv = int(k.shape[1]) if (k is not None and hasattr(k, "shape") and k.dim() == 4) else 0
     return FaParams(q=_ptr(q), k=_ptr(k), v=_ptr(v), o=_ptr(o), lse=_ptr(lse), k_len=_ptr(k_len),
                     dev_status=_ptr(dev_status), B=B, H=H, N=N, d=d, causal=int(bool(causal)),
-                    scale=float(scale), o_dtype=o_dtype, flags=int(flags), timeout_ms=int(timeout_ms))
+                    scale=float(scale), o_dtype=o_dtype, flags=int(flags), timeout_ms=int(timeout_ms),
+                    H_kv=H_kv)
 
 
 def fa_fwd_ex(q, k, v, o, lse, causal: bool, scale: float, k_len=None, dev_status=None, flags: int = 0,
               timeout_ms: int = 0, stream=None):
     """fa_fwd_ex: as fa_fwd, plus k_len (int32 [B] CUDA tensor), o may be bf16,
-    an optional int32 status word, FA_FLAG_* flags and the wait time limit."""
+    an optional int32 status word, FA_FLAG_* flags and the wait time limit.
+    k and v may have fewer heads than q ([B, H_kv, N, d], H_kv dividing H)."""
     p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms)
     _check(load().fa_fwd_ex(ctypes.byref(p), _stream(stream)), "fa_fwd_ex")
 

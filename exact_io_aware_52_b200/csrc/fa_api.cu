@@ -87,6 +87,7 @@ fa_status validate(const fa_fwd_params *p) {
     if (p->causal != 0 && p->causal != 1) return FA_ERR_INVALID_ARGUMENT;
     if (p->o_dtype != FA_O_F32 && p->o_dtype != FA_O_BF16) return FA_ERR_INVALID_ARGUMENT;
     if (p->flags & ~FA_FLAG_EAGER_RESCALE) return FA_ERR_INVALID_ARGUMENT;
+    if (p->H_kv < 0 || (p->H_kv > 0 && p->H % p->H_kv != 0)) return FA_ERR_INVALID_ARGUMENT;
     if (p->d != 64 && p->d != 128) return FA_ERR_UNSUPPORTED;
     const long long rows = (long long)p->B * p->H * p->N;
     if (rows == 0) return FA_OK;
@@ -138,15 +139,18 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     fa::FwdParams kp;
     std::memset(&kp, 0, sizeof kp);
     const int BH = p->B * p->H;
+    const int H_kv = p->H_kv > 0 ? p->H_kv : p->H;
     if ((st = encode_map(&kp.tm_q, p->q, BH, p->N, p->d)) != FA_OK) return st;
-    if ((st = encode_map(&kp.tm_k, p->k, BH, p->N, p->d)) != FA_OK) return st;
-    if ((st = encode_map(&kp.tm_v, p->v, BH, p->N, p->d)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_k, p->k, p->B * H_kv, p->N, p->d)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_v, p->v, p->B * H_kv, p->N, p->d)) != FA_OK) return st;
     kp.o = p->o;
     kp.lse = p->lse;
     kp.k_len = p->k_len;
     kp.status = p->dev_status;
     kp.B = p->B;
     kp.H = p->H;
+    kp.group = p->H / H_kv;
+    kp.H_kv = H_kv;
     kp.N = p->N;
     kp.n_blocks = (p->N + fa::kUnitRows - 1) / fa::kUnitRows;
     kp.n_units = BH * kp.n_blocks;
@@ -191,11 +195,12 @@ fa_status fa_fwd_host(const fa_fwd_host_params *hp, void *stream) {
     if (!hp->q || !hp->k || !hp->v || !hp->o || !hp->lse) return FA_ERR_INVALID_ARGUMENT;
     if ((hp->k_len == nullptr) != (p->k_len == nullptr)) return FA_ERR_INVALID_ARGUMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const size_t in_bytes = rows * p->d * 2;
+    const size_t q_bytes = rows * p->d * 2;
+    const size_t kv_bytes = (size_t)p->B * (p->H_kv > 0 ? p->H_kv : p->H) * p->N * p->d * 2;
     const size_t o_bytes = rows * p->d * (p->o_dtype == FA_O_BF16 ? 2 : 4);
-    if (cudaMemcpyAsync(const_cast<void *>(p->q), hp->q, in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(const_cast<void *>(p->k), hp->k, in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(const_cast<void *>(p->v), hp->v, in_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    if (cudaMemcpyAsync(const_cast<void *>(p->q), hp->q, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(const_cast<void *>(p->k), hp->k, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(const_cast<void *>(p->v), hp->v, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return FA_ERR_CUDA;
     if (hp->k_len && cudaMemcpyAsync(const_cast<int32_t *>(p->k_len), hp->k_len, sizeof(int32_t) * p->B,
                                      cudaMemcpyHostToDevice, s) != cudaSuccess)

@@ -82,12 +82,15 @@ __device__ __forceinline__ uint32_t col_s(uint32_t x) { return x * 128u; }      
 __device__ __forceinline__ uint32_t col_o(uint32_t x, uint32_t d) { return 256u + x * d; }  // O_X
 
 struct FwdParams {
-    CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps over [B*H][N][D] bf16; box {64, 128, 1}; 128-byte swizzle
+    CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps over [B*H][N][D] (Q) and [B*H_kv][N][D] (K, V) bf16;
+                                   // box {64, 128, 1}; 128-byte swizzle
     void *o;                       // [B, H, N, D] fp32 or bf16
     float *lse;                    // [B, H, N]
     const int32_t *k_len;          // [B] or nullptr
     int32_t *status;               // device status word or nullptr
     int B, H, N;
+    int H_kv;                      // key/value heads; query head h uses key/value head h / group
+    int group;                     // H / H_kv
     int n_blocks;                  // ceil(N / 256)
     int n_units;                   // B * H * n_blocks
     int causal;
@@ -131,6 +134,7 @@ struct Cfg {
 
 struct UnitCoord {
     int bh, b, blk;
+    int bh_kv;  // key/value head row of K and V: b * H_kv + h / group
     int n[2];  // key tiles of query tile A and B (a prefix [0, n) of the key tiles)
     int nmax;
 };
@@ -150,6 +154,7 @@ __device__ __forceinline__ UnitCoord decode_unit(const FwdParams &p, int t) {
     u.blk = p.n_blocks - 1 - t % p.n_blocks;
     u.bh = t / p.n_blocks;
     u.b = u.bh / p.H;
+    u.bh_kv = u.b * p.H_kv + (u.bh - u.b * p.H) / p.group;
     int kv_lim = p.N;
     if (p.k_len) kv_lim = min(max(__ldg(p.k_len + u.b), 0), p.N);
 #pragma unroll
@@ -515,7 +520,7 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_3d(sK + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_k, &bars[C::kBarKFull + slot],
-                                c * 64, j * BN, u.bh);
+                                c * 64, j * BN, u.bh_kv);
                 ++gk;
             }
             {
@@ -528,7 +533,7 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_3d(sV + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_v, &bars[C::kBarVFull + slot],
-                                c * 64, j * BN, u.bh);
+                                c * 64, j * BN, u.bh_kv);
                 ++gv;
             }
         }

@@ -31,6 +31,7 @@ class Workload:
     qk_std: float = 1.0
     kpad: tuple | None = None          # (lo, hi) inclusive range of key lengths, or None
     sample_rows_per_head: int | None = None  # rows the oracle checks per head (None: all)
+    H_kv: int | None = None            # key/value heads (grouped attention); None: H
     seed: int = 0
     notes: str = field(default="", compare=False)
 
@@ -38,6 +39,10 @@ class Workload:
     def scale(self) -> float:
         # the float32 value the kernel receives, as a Python float
         return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32).item())
+
+    @property
+    def kv_heads(self) -> int:
+        return self.H if self.H_kv is None else self.H_kv
 
     def flops(self) -> float:
         """Nominal attention FLOPs: 4*B*H*N^2*d, halved when causal."""
@@ -55,21 +60,25 @@ WORKLOADS = {
                 sample_rows_per_head=512, seed=52004),
     5: Workload("softmax-stress causal B1 H16 N65536 d128 QK~N(0,4^2)", 1, 16, 65536, 128, True,
                 qk_std=4.0, sample_rows_per_head=256, seed=52005),
+    # grouped key/value heads (multi-query family): 8 key/value heads serve 32 query heads
+    6: Workload("long-context causal grouped-KV B1 H32 Hkv8 N16384 d128", 1, 32, 16384, 128, True,
+                sample_rows_per_head=128, seed=52006, H_kv=8),
 }
 
 
 def make_inputs(w: Workload, seed: int | None = None):
     """Draw (q, k, v, k_len) on the CPU for workload ``w``.
 
-    q, k, v: bfloat16 [B, H, N, d] contiguous CPU tensors.
+    q: bfloat16 [B, H, N, d]; k, v: bfloat16 [B, H_kv, N, d] contiguous CPU tensors.
     k_len: int32 [B] CPU tensor, or None when the workload has no key padding.
     """
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed if seed is None else seed)
     shape = (w.B, w.H, w.N, w.d)
+    kv_shape = (w.B, w.kv_heads, w.N, w.d)
     q = (torch.randn(shape, generator=g, dtype=torch.float32) * w.qk_std).to(torch.bfloat16)
-    k = (torch.randn(shape, generator=g, dtype=torch.float32) * w.qk_std).to(torch.bfloat16)
-    v = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k = (torch.randn(kv_shape, generator=g, dtype=torch.float32) * w.qk_std).to(torch.bfloat16)
+    v = torch.randn(kv_shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
     k_len = None
     if w.kpad is not None:
         lo, hi = w.kpad
@@ -98,6 +107,6 @@ def sample_rows(w: Workload, seed: int | None = None):
     return np.concatenate(out)
 
 
-def custom(B, H, N, d, causal, qk_std=1.0, kpad=None, seed=1, name="custom") -> Workload:
+def custom(B, H, N, d, causal, qk_std=1.0, kpad=None, seed=1, name="custom", H_kv=None) -> Workload:
     """A workload of arbitrary shape (tests of ragged and edge shapes)."""
-    return Workload(name, B, H, N, d, causal, qk_std=qk_std, kpad=kpad, seed=seed)
+    return Workload(name, B, H, N, d, causal, qk_std=qk_std, kpad=kpad, seed=seed, H_kv=H_kv)

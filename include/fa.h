@@ -15,7 +15,10 @@
  * unico kernel de CUDA"): no N x N buffer, no workspace of any kind.
  *
  * Layout (all tensors contiguous, row-major):
- *   q, k, v : bf16  [B, H, N, d]      (one N x d matrix per (b, h))
+ *   q       : bf16  [B, H, N, d]      (one N x d matrix per (b, h))
+ *   k, v    : bf16  [B, H_kv, N, d]   (fa_fwd: H_kv = H; fa_fwd_ex may group:
+ *             query head h attends with key/value head h / (H / H_kv), the
+ *             multi-query attention of section "FlashAttention-2 (2023)")
  *   o       : fp32  [B, H, N, d]  (fa_fwd; fa_fwd_ex may select bf16)
  *   lse     : fp32  [B, H, N]
  *   k_len   : int32 [B]  (fa_fwd_ex only; key j of batch b is masked iff
@@ -85,7 +88,7 @@ FA_EXPORT fa_status fa_fwd(const void *q, const void *k, const void *v, float *o
                  int B, int H, int N, int d, int causal, float scale, void *stream);
 
 typedef struct {
-    const void *q, *k, *v;   /* device bf16 [B, H, N, d]                              */
+    const void *q, *k, *v;   /* device bf16: q [B, H, N, d]; k, v [B, H_kv, N, d]     */
     void *o;                 /* device [B, H, N, d], fp32 or bf16 per o_dtype         */
     float *lse;              /* device fp32 [B, H, N]                                 */
     const int32_t *k_len;    /* device int32 [B], or NULL (no key padding)           */
@@ -98,6 +101,8 @@ typedef struct {
     int o_dtype;             /* fa_o_dtype                                            */
     int flags;               /* FA_FLAG_* bits, 0 by default                          */
     uint32_t timeout_ms;     /* per-wait time limit on the device; 0 = 2000 ms        */
+    int H_kv;                /* key/value heads (k, v are [B, H_kv, N, d]); 0 means H;
+                                must divide H (1 = multi-query attention)             */
 } fa_fwd_params;
 
 /*
@@ -109,7 +114,7 @@ typedef struct {
 FA_EXPORT fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream);
 
 typedef struct {
-    const void *q, *k, *v;   /* host bf16 [B, H, N, d] (pinned memory for async copies) */
+    const void *q, *k, *v;   /* host bf16, shapes as in dev (pinned for async copies) */
     const int32_t *k_len;    /* host int32 [B] or NULL                                */
     void *o;                 /* host output, dtype per dev.o_dtype                    */
     float *lse;              /* host fp32 [B, H, N]                                   */

@@ -54,7 +54,7 @@ def load_library(path: str):
     f = lib.attn_oracle_f64
     f.restype = ctypes.c_int
     f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                  ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                   ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
                   ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     return lib
@@ -84,7 +84,8 @@ def attention_f64(q, k, v, causal: bool, scale: float, k_len=None, rows=None,
                   nthreads: int | None = None, lib=None):
     """Exact attention in fp64 from bf16 inputs.
 
-    q, k, v: [B, H, N, d] bf16 (torch CPU tensor or uint16 bit array).
+    q: [B, H, N, d] and k, v: [B, H_kv, N, d] bf16 (torch CPU tensors or uint16
+    bit arrays); H_kv divides H and query head h uses key/value head h // (H // H_kv).
     causal: key j is masked for query i when j > i.
     scale: the float32 multiplier of q.k (the definition's 1/sqrt(d_k)).
     k_len: None or int sequence of length B; key j of batch b masked iff j >= k_len[b].
@@ -94,9 +95,12 @@ def attention_f64(q, k, v, causal: bool, scale: float, k_len=None, rows=None,
     rows is None (row r = (b*H + h)*N + i).
     """
     qb, kb, vb = _as_bf16_bits(q), _as_bf16_bits(k), _as_bf16_bits(v)
-    if qb.ndim != 4 or qb.shape != kb.shape or qb.shape != vb.shape:
-        raise ValueError("q, k, v must share one [B, H, N, d] shape")
+    if qb.ndim != 4 or kb.ndim != 4 or kb.shape != vb.shape:
+        raise ValueError("q must be [B, H, N, d] and k, v [B, H_kv, N, d]")
     B, H, N, d = qb.shape
+    H_kv = kb.shape[1]
+    if (kb.shape[0], kb.shape[2], kb.shape[3]) != (B, N, d) or H_kv == 0 or H % H_kv:
+        raise ValueError("k, v must be [B, H_kv, N, d] with H_kv dividing H")
     kl = None
     if k_len is not None:
         kl = np.ascontiguousarray(np.asarray(k_len, dtype=np.int32).reshape(-1))
@@ -114,7 +118,7 @@ def attention_f64(q, k, v, causal: bool, scale: float, k_len=None, rows=None,
     lib = _load() if lib is None else lib
     rc = lib.attn_oracle_f64(
         qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
-        None if kl is None else kl.ctypes.data, B, H, N, d, int(bool(causal)),
+        None if kl is None else kl.ctypes.data, B, H, H_kv, N, d, int(bool(causal)),
         ctypes.c_float(scale), None if rr is None else rr.ctypes.data,
         n_rows, o.ctypes.data, lse.ctypes.data, int(nt))
     if rc != 0:

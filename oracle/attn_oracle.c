@@ -22,6 +22,11 @@
  *   5. O_i = sum_j p_j v_j and lse_i = m + ln l (natural log of
  *      sum_j exp(s_j) over A_i).  An empty A_i gives O_i = 0, lse_i = -inf.
  *
+ * Grouped keys and values (the multi-query attention that section
+ * "FlashAttention-2 (2023)" says the method was extended to): with H_kv
+ * key/value heads, query head h attends with key/value head h / (H / H_kv);
+ * H_kv = H is ordinary multi-head attention, H_kv = 1 multi-query attention.
+ *
  * There is no tiling, no online recurrence and no reordering beyond this
  * definition: one score row at a time, in key order.
  */
@@ -42,7 +47,8 @@ static double bf16_bits_to_double(uint16_t bits) {
 
 /*
  * attn_oracle_f64
- *   q, k, v : bf16 bit patterns, contiguous [B, H, N, d]
+ *   q       : bf16 bit patterns, contiguous [B, H, N, d]
+ *   k, v    : bf16 bit patterns, contiguous [B, H_kv, N, d]; H_kv divides H
  *   k_len   : NULL, or int32[B]; key j of batch b is masked iff j >= k_len[b]
  *             (values outside [0, N] are clamped to it)
  *   causal  : nonzero masks key j for query i when j > i
@@ -55,10 +61,11 @@ static double bf16_bits_to_double(uint16_t bits) {
  * Returns 0, or -1 on a bad argument, -2 on allocation failure.
  */
 int attn_oracle_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                    const int32_t *k_len, int B, int H, int N, int d,
+                    const int32_t *k_len, int B, int H, int H_kv, int N, int d,
                     int causal, float scale, const int64_t *rows,
                     int64_t n_rows, double *o, double *lse, int nthreads) {
     if (B < 0 || H < 0 || N < 0 || d <= 0) return -1;
+    if (H_kv <= 0 || H % H_kv != 0) return -1;
     if (!q || !k || !v || !o || !lse) return (n_rows == 0) ? 0 : -1;
     const int64_t total_rows = (int64_t)B * H * N;
     if (!rows) n_rows = total_rows;
@@ -87,6 +94,8 @@ int attn_oracle_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             const int64_t bh = r / N;
             const int i = (int)(r % N);
             const int b = (int)(bh / H);
+            const int h = (int)(bh % H);
+            const int64_t bh_kv = (int64_t)b * H_kv + h / (H / H_kv); /* this head's key/value head */
             int L = N;
             if (k_len) {
                 L = k_len[b];
@@ -94,8 +103,8 @@ int attn_oracle_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 if (L > N) L = N;
             }
             const uint16_t *qi = q + r * d;
-            const uint16_t *kb = k + bh * (int64_t)N * d;
-            const uint16_t *vb = v + bh * (int64_t)N * d;
+            const uint16_t *kb = k + bh_kv * (int64_t)N * d;
+            const uint16_t *vb = v + bh_kv * (int64_t)N * d;
             double *oi = o + t * d;
 
             /* step 1-2: widened query row, full score row over every key */

@@ -272,6 +272,35 @@ def pin_row_subset(lib):
     np.testing.assert_array_equal(lse_s, lse.reshape(-1)[rows])
 
 
+def pin_grouped_heads(lib):
+    """Grouped key/value heads: against torch's float64 scaled_dot_product_attention
+    with enable_gqa (a library routine), and equal to multi-head attention on K, V
+    with each key/value head repeated H / H_kv times; H_kv = 1 is multi-query."""
+    g = torch.Generator().manual_seed(22)
+    B, H, N, d = 2, 6, 23, 8
+    for H_kv in (1, 2, 3):
+        q = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+        k = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
+        v = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
+        for causal, k_len in ((False, None), (True, [20, 9])):
+            o, lse = run(lib, q, k, v, causal, 0.35, k_len=k_len)
+            rep = H // H_kv
+            o_mha, lse_mha = run(lib, q, k.repeat_interleave(rep, dim=1), v.repeat_interleave(rep, dim=1),
+                                 causal, 0.35, k_len=k_len)
+            np.testing.assert_array_equal(o, o_mha)
+            np.testing.assert_array_equal(lse, lse_mha)
+            scale = float(np.float32(0.35))
+            mask = torch.ones(B, 1, N, N, dtype=torch.bool)
+            if causal:
+                mask &= torch.ones(N, N, dtype=torch.bool).tril()
+            if k_len is not None:
+                for b in range(B):
+                    mask[b, :, :, k_len[b]:] = False
+            o_ref = torch.nn.functional.scaled_dot_product_attention(
+                q.double(), k.double(), v.double(), attn_mask=mask, scale=scale, enable_gqa=True)
+            np.testing.assert_allclose(o, o_ref.numpy(), rtol=1e-10, atol=1e-11)
+
+
 ALL_PINS = [pin_zero_query_means, pin_dominant_key, pin_library_sdpa, pin_permutation_invariance,
             pin_single_key, pin_constant_values, pin_rows_are_distributions, pin_convex_hull,
-            pin_online_equals_two_pass, pin_large_logits, pin_row_subset]
+            pin_online_equals_two_pass, pin_large_logits, pin_row_subset, pin_grouped_heads]

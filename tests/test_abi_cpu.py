@@ -48,7 +48,7 @@ def test_status_strings_and_version():
 
 def _params(**kw):
     base = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0x50000, k_len=None, dev_status=None,
-                B=1, H=2, N=128, d=64, causal=0, scale=0.125, o_dtype=0, flags=0, timeout_ms=0)
+                B=1, H=2, N=128, d=64, causal=0, scale=0.125, o_dtype=0, flags=0, timeout_ms=0, H_kv=0)
     base.update(kw)
     return fb.FaParams(**base)
 
@@ -74,6 +74,9 @@ def _ex(**kw):
     (dict(causal=2), fb.FA_ERR_INVALID_ARGUMENT),
     (dict(o_dtype=7), fb.FA_ERR_INVALID_ARGUMENT),
     (dict(flags=0x80), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(H_kv=-1), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(H=6, H_kv=4), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(H=6, H_kv=7), fb.FA_ERR_INVALID_ARGUMENT),
     (dict(d=32), fb.FA_ERR_UNSUPPORTED),
     (dict(d=256), fb.FA_ERR_UNSUPPORTED),
     (dict(d=96), fb.FA_ERR_UNSUPPORTED),

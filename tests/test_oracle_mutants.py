@@ -22,8 +22,8 @@ MUTANTS = [
     ("output sums K instead of V", [("const uint16_t *vj = vb + (int64_t)j * d;",
                                      "const uint16_t *vj = kb + (int64_t)j * d;")]),
     ("softmax not normalised", [("const double p = s[j] / l;", "const double p = s[j];")]),
-    ("transposed scores", [("const uint16_t *qi = q + r * d;", "const uint16_t *qi = k + r * d;"),
-                           ("const uint16_t *kb = k + bh * (int64_t)N * d;",
+    ("transposed scores", [("const uint16_t *qi = q + r * d;", "const uint16_t *qi = k + (bh_kv * N + i) * d;"),
+                           ("const uint16_t *kb = k + bh_kv * (int64_t)N * d;",
                             "const uint16_t *kb = q + bh * (int64_t)N * d;")]),
     ("no max subtraction", [("s[j] = exp(s[j] - m);", "s[j] = exp(s[j]);"),
                             ("lse[t] = m + log(l);", "lse[t] = log(l);")]),
@@ -32,6 +32,7 @@ MUTANTS = [
     ("last allowed key dropped", [("for (int j = 0; j < allowed_end; ++j) {\n                const double p",
                                    "for (int j = 0; j < allowed_end - 1; ++j) {\n                const double p")]),
     ("empty row gives zero lse", [("lse[t] = -INFINITY;", "lse[t] = 0.0;")]),
+    ("grouped head taken modulo", [("h / (H / H_kv);", "h % H_kv;")]),
 ]
 
 

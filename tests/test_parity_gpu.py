@@ -25,7 +25,7 @@ def rand_inputs(B, H, N, d, seed, std=1.0):
 
 
 # ------------------------------------------------------------ the five workloads
-@pytest.mark.parametrize("wid", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("wid", [1, 2, 3, 4, 5, 6])
 def test_workload_parity(wid):
     """Each seeded workload at its full size, in the launch configuration the
     benchmark times (all rows for 1-3, the seeded row sample for 4-5)."""
@@ -61,6 +61,26 @@ def test_key_padding_edges(d, causal):
     k_len = [0, 1, N - 1, N, N + 50, -5, 128, 129]
     q, k, v = rand_inputs(len(k_len), 2, N, d, seed=31 + d + causal)
     check_case(q, k, v, causal, 1.0 / math.sqrt(d), k_len=k_len)
+
+
+# ------------------------------------------------------------ grouped key/value heads
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H_kv", [1, 2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_grouped_kv_heads(d, H_kv, causal):
+    """Query head h attends with key/value head h // (H // H_kv); H_kv = 1 is
+    multi-query attention."""
+    B, H, N = 2, 8, 333
+    g = torch.Generator().manual_seed(40 + d + H_kv + causal)
+    q = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
+    check_case(q, k, v, causal, 1.0 / math.sqrt(d), k_len=[333, 201])
+    # the same arithmetic as multi-head attention on repeated key/value heads: bit-identical
+    o1, l1 = run_gpu(q, k, v, causal, 1.0 / math.sqrt(d))
+    o2, l2 = run_gpu(q, k.repeat_interleave(H // H_kv, dim=1), v.repeat_interleave(H // H_kv, dim=1), causal,
+                     1.0 / math.sqrt(d))
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
 # ------------------------------------------------------------ closed forms on the GPU

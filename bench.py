@@ -185,17 +185,26 @@ def dist_setup(args):
     return world, rank, local
 
 
+def workload_config(w, world: int, q_bytes: int) -> dict:
+    """The `config` object of the JSON line (identical for both arms)."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "N": w.N, "d": w.d,
+            "causal": w.causal, "out": "fp32 O + fp32 lse", "flops_per_step_per_gpu": w.flops(),
+            "l2": "inputs larger than L2 (Q,K,V %.0f MB > 126 MB); no flush" % (q_bytes / 1e6),
+            "parallelism": f"replicas x{world}"}
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """Largest value of x over all ranks (the timing rule: the slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -269,11 +278,10 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-                   "step": f"fp64 CPU oracle on {rows_per_step} sampled query rows"},
+        "config": workload_config(w, world, (q.numel() + k.numel() + v.numel()) * 2),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{rows_per_step} uniformly sampled query rows per step, "
-                                   f"{args.steps} steps"},
+                         "sample": f"each step: the fp64 oracle on {rows_per_step} uniformly sampled query "
+                                   f"rows of the workload (all keys of each row); {args.steps} steps"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -382,11 +390,7 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "N": w.N, "d": w.d,
-                   "causal": w.causal, "out": "fp32 O + fp32 lse", "flops_per_step_per_gpu": flops,
-                   "l2": "inputs larger than L2 (Q,K,V %.0f MB > 126 MB); no flush"
-                         % ((q.numel() + k.numel() + v.numel()) * 2 / 1e6),
-                   "parallelism": f"replicas x{world}"},
+        "config": workload_config(w, world, (q.numel() + k.numel() + v.numel()) * 2),
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": roofline,
         "cpu_baseline": cpu,

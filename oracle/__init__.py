@@ -54,7 +54,7 @@ def load_library(path: str):
     f = lib.attn_oracle_f64
     f.restype = ctypes.c_int
     f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                  ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                   ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
                   ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     return lib
@@ -84,8 +84,9 @@ def attention_f64(q, k, v, causal: bool, scale: float, k_len=None, rows=None,
                   nthreads: int | None = None, lib=None):
     """Exact attention in fp64 from bf16 inputs.
 
-    q: [B, H, N, d] and k, v: [B, H_kv, N, d] bf16 (torch CPU tensors or uint16
-    bit arrays); H_kv divides H and query head h uses key/value head h // (H // H_kv).
+    q: [B, H, N, d] and k, v: [B, H_kv, Nk, d] bf16 (torch CPU tensors or uint16
+    bit arrays); H_kv divides H and query head h uses key/value head h // (H // H_kv);
+    with Nk keys query i sits at key position i + Nk - N (causal: key j <= i + Nk - N).
     causal: key j is masked for query i when j > i.
     scale: the float32 multiplier of q.k (the definition's 1/sqrt(d_k)).
     k_len: None or int sequence of length B; key j of batch b masked iff j >= k_len[b].
@@ -98,9 +99,9 @@ def attention_f64(q, k, v, causal: bool, scale: float, k_len=None, rows=None,
     if qb.ndim != 4 or kb.ndim != 4 or kb.shape != vb.shape:
         raise ValueError("q must be [B, H, N, d] and k, v [B, H_kv, N, d]")
     B, H, N, d = qb.shape
-    H_kv = kb.shape[1]
-    if (kb.shape[0], kb.shape[2], kb.shape[3]) != (B, N, d) or H_kv == 0 or H % H_kv:
-        raise ValueError("k, v must be [B, H_kv, N, d] with H_kv dividing H")
+    H_kv, Nk = kb.shape[1], kb.shape[2]
+    if (kb.shape[0], kb.shape[3]) != (B, d) or H_kv == 0 or H % H_kv:
+        raise ValueError("k, v must be [B, H_kv, Nk, d] with H_kv dividing H")
     kl = None
     if k_len is not None:
         kl = np.ascontiguousarray(np.asarray(k_len, dtype=np.int32).reshape(-1))
@@ -118,7 +119,7 @@ def attention_f64(q, k, v, causal: bool, scale: float, k_len=None, rows=None,
     lib = _load() if lib is None else lib
     rc = lib.attn_oracle_f64(
         qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
-        None if kl is None else kl.ctypes.data, B, H, H_kv, N, d, int(bool(causal)),
+        None if kl is None else kl.ctypes.data, B, H, H_kv, N, Nk, d, int(bool(causal)),
         ctypes.c_float(scale), None if rr is None else rr.ctypes.data,
         n_rows, o.ctypes.data, lse.ctypes.data, int(nt))
     if rc != 0:

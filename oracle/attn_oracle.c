@@ -22,6 +22,11 @@
  *   5. O_i = sum_j p_j v_j and lse_i = m + ln l (natural log of
  *      sum_j exp(s_j) over A_i).  An empty A_i gives O_i = 0, lse_i = -inf.
  *
+ * Queries and keys may differ in number (N_q queries against N_k keys, the
+ * cached-keys setting of section "Soluciones especializadas"): query i then
+ * sits at key position i + N_k - N_q, and the causal mask allows key j iff
+ * j <= i + N_k - N_q (with N_q = N_k this is j <= i).
+ *
  * Grouped keys and values (the multi-query attention that section
  * "FlashAttention-2 (2023)" says the method was extended to): with H_kv
  * key/value heads, query head h attends with key/value head h / (H / H_kv);
@@ -47,11 +52,11 @@ static double bf16_bits_to_double(uint16_t bits) {
 
 /*
  * attn_oracle_f64
- *   q       : bf16 bit patterns, contiguous [B, H, N, d]
- *   k, v    : bf16 bit patterns, contiguous [B, H_kv, N, d]; H_kv divides H
+ *   q       : bf16 bit patterns, contiguous [B, H, N, d]   (N queries)
+ *   k, v    : bf16 bit patterns, contiguous [B, H_kv, Nk, d] (Nk keys); H_kv divides H
  *   k_len   : NULL, or int32[B]; key j of batch b is masked iff j >= k_len[b]
  *             (values outside [0, N] are clamped to it)
- *   causal  : nonzero masks key j for query i when j > i
+ *   causal  : nonzero masks key j for query i when j > i + Nk - N
  *   scale   : the float multiplier applied to q.k (1/sqrt(d_k) in the
  *             definition); widened to double
  *   rows    : NULL (every row, in order) or n_rows flat row ids
@@ -61,11 +66,12 @@ static double bf16_bits_to_double(uint16_t bits) {
  * Returns 0, or -1 on a bad argument, -2 on allocation failure.
  */
 int attn_oracle_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                    const int32_t *k_len, int B, int H, int H_kv, int N, int d,
+                    const int32_t *k_len, int B, int H, int H_kv, int N, int Nk, int d,
                     int causal, float scale, const int64_t *rows,
                     int64_t n_rows, double *o, double *lse, int nthreads) {
     if (B < 0 || H < 0 || N < 0 || d <= 0) return -1;
     if (H_kv <= 0 || H % H_kv != 0) return -1;
+    if (Nk < 0) return -1;
     if (!q || !k || !v || !o || !lse) return (n_rows == 0) ? 0 : -1;
     const int64_t total_rows = (int64_t)B * H * N;
     if (!rows) n_rows = total_rows;
@@ -76,7 +82,7 @@ int attn_oracle_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 
 #pragma omp parallel num_threads(nt)
     {
-        double *s = (double *)malloc(sizeof(double) * (N > 0 ? (size_t)N : 1));
+        double *s = (double *)malloc(sizeof(double) * (Nk > 0 ? (size_t)Nk : 1));
         double *qrow = (double *)malloc(sizeof(double) * (size_t)d);
         if (!s || !qrow) {
 #pragma omp atomic write
@@ -96,20 +102,20 @@ int attn_oracle_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             const int b = (int)(bh / H);
             const int h = (int)(bh % H);
             const int64_t bh_kv = (int64_t)b * H_kv + h / (H / H_kv); /* this head's key/value head */
-            int L = N;
+            int L = Nk;
             if (k_len) {
                 L = k_len[b];
                 if (L < 0) L = 0;
-                if (L > N) L = N;
+                if (L > Nk) L = Nk;
             }
             const uint16_t *qi = q + r * d;
-            const uint16_t *kb = k + bh_kv * (int64_t)N * d;
-            const uint16_t *vb = v + bh_kv * (int64_t)N * d;
+            const uint16_t *kb = k + bh_kv * (int64_t)Nk * d;
+            const uint16_t *vb = v + bh_kv * (int64_t)Nk * d;
             double *oi = o + t * d;
 
             /* step 1-2: widened query row, full score row over every key */
             for (int c = 0; c < d; ++c) qrow[c] = bf16_bits_to_double(qi[c]);
-            for (int j = 0; j < N; ++j) {
+            for (int j = 0; j < Nk; ++j) {
                 const uint16_t *kj = kb + (int64_t)j * d;
                 double acc = 0.0;
                 for (int c = 0; c < d; ++c) acc += qrow[c] * bf16_bits_to_double(kj[c]);
@@ -117,7 +123,8 @@ int attn_oracle_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             }
             /* step 3: allowed set A_i */
             int allowed_end = L;                    /* keys [0, L) survive padding */
-            if (causal && i + 1 < allowed_end) allowed_end = i + 1; /* j <= i */
+            if (causal && (int64_t)i + 1 + Nk - N < allowed_end)
+                allowed_end = (int)((int64_t)i + 1 + Nk - N);      /* j <= i + Nk - N */
             /* step 4: max-subtracted softmax over A_i = [0, allowed_end) */
             if (allowed_end <= 0) {
                 for (int c = 0; c < d; ++c) oi[c] = 0.0;

@@ -301,6 +301,36 @@ def pin_grouped_heads(lib):
             np.testing.assert_allclose(o, o_ref.numpy(), rtol=1e-10, atol=1e-11)
 
 
+def pin_fewer_queries_than_keys(lib):
+    """N_q queries against N_k > N_q keys: against torch's float64
+    scaled_dot_product_attention with the bottom-right causal mask (key j
+    allowed for query i iff j <= i + N_k - N_q), and equal to the last N_q
+    rows of the square problem whose last N_q query rows are these queries."""
+    g = torch.Generator().manual_seed(23)
+    B, H, Nq, Nk, d = 2, 2, 7, 30, 8
+    q = torch.randn(B, H, Nq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, H, Nk, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, Nk, d, generator=g).to(torch.bfloat16)
+    scale = float(np.float32(0.4))
+    for causal, k_len in ((False, None), (True, None), (True, [27, 30])):
+        o, lse = run(lib, q, k, v, causal, 0.4, k_len=k_len)
+        mask = torch.ones(B, 1, Nq, Nk, dtype=torch.bool)
+        if causal:
+            mask &= torch.ones(Nq, Nk, dtype=torch.bool).tril(diagonal=Nk - Nq)
+        if k_len is not None:
+            for b in range(B):
+                mask[b, :, :, k_len[b]:] = False
+        o_ref = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double(),
+                                                                 attn_mask=mask, scale=scale)
+        np.testing.assert_allclose(o, o_ref.numpy(), rtol=1e-10, atol=1e-11)
+        qfull = torch.randn(B, H, Nk, d, generator=g).to(torch.bfloat16)
+        qfull[:, :, Nk - Nq:] = q
+        o_sq, lse_sq = run(lib, qfull, k, v, causal, 0.4, k_len=k_len)
+        np.testing.assert_array_equal(o, o_sq[:, :, Nk - Nq:])
+        np.testing.assert_array_equal(lse, lse_sq[:, :, Nk - Nq:])
+
+
 ALL_PINS = [pin_zero_query_means, pin_dominant_key, pin_library_sdpa, pin_permutation_invariance,
             pin_single_key, pin_constant_values, pin_rows_are_distributions, pin_convex_hull,
-            pin_online_equals_two_pass, pin_large_logits, pin_row_subset, pin_grouped_heads]
+            pin_online_equals_two_pass, pin_large_logits, pin_row_subset, pin_grouped_heads,
+            pin_fewer_queries_than_keys]

@@ -12,8 +12,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")
 
 # (name, [(original text, mistaken text), ...])
 MUTANTS = [
-    ("causal mask off by one", [("if (causal && i + 1 < allowed_end) allowed_end = i + 1;",
-                                 "if (causal && i < allowed_end) allowed_end = i;")]),
+    ("causal mask off by one", [("(int64_t)i + 1 + Nk - N < allowed_end)\n                allowed_end = (int)((int64_t)i + 1 + Nk - N);",
+                                 "(int64_t)i + Nk - N < allowed_end)\n                allowed_end = (int)((int64_t)i + Nk - N);")]),
     ("scale dropped", [("s[j] = sigma * acc;", "s[j] = acc;")]),
     ("scale applied twice", [("s[j] = sigma * acc;", "s[j] = sigma * sigma * acc;")]),
     ("max missing from lse", [("lse[t] = m + log(l);", "lse[t] = log(l);")]),
@@ -22,9 +22,11 @@ MUTANTS = [
     ("output sums K instead of V", [("const uint16_t *vj = vb + (int64_t)j * d;",
                                      "const uint16_t *vj = kb + (int64_t)j * d;")]),
     ("softmax not normalised", [("const double p = s[j] / l;", "const double p = s[j];")]),
-    ("transposed scores", [("const uint16_t *qi = q + r * d;", "const uint16_t *qi = k + (bh_kv * N + i) * d;"),
-                           ("const uint16_t *kb = k + bh_kv * (int64_t)N * d;",
-                            "const uint16_t *kb = q + bh * (int64_t)N * d;")]),
+    # query row i taken from K and key j from Q (j wrapped into the query range so the
+    # mistaken reads stay inside the buffers): the transposed score matrix when N_q = N_k
+    ("transposed scores", [("const uint16_t *qi = q + r * d;", "const uint16_t *qi = k + (bh_kv * Nk + i) * d;"),
+                           ("const uint16_t *kj = kb + (int64_t)j * d;",
+                            "const uint16_t *kj = q + (bh * N + j % N) * d;")]),
     ("no max subtraction", [("s[j] = exp(s[j] - m);", "s[j] = exp(s[j]);"),
                             ("lse[t] = m + log(l);", "lse[t] = log(l);")]),
     ("sign of dot product", [("acc += qrow[c] *", "acc -= qrow[c] *")]),
@@ -33,6 +35,7 @@ MUTANTS = [
                                    "for (int j = 0; j < allowed_end - 1; ++j) {\n                const double p")]),
     ("empty row gives zero lse", [("lse[t] = -INFINITY;", "lse[t] = 0.0;")]),
     ("grouped head taken modulo", [("h / (H / H_kv);", "h % H_kv;")]),
+    ("causal diagonal not shifted", [("allowed_end = (int)((int64_t)i + 1 + Nk - N);", "allowed_end = i + 1;")]),
 ]
 
 

@@ -99,7 +99,7 @@ def algorithmic_bytes(w, k_len) -> float:
     """Compulsory HBM bytes of one launch: Q, K, V read once (valid keys only
     under key padding), O (fp32) and lse written once."""
     n_elem = w.B * w.H * w.N * w.d
-    kv_rows = w.kv_heads * (sum(min(max(int(x), 0), w.N) for x in k_len) if k_len is not None else w.B * w.N)
+    kv_rows = w.kv_heads * (sum(min(max(int(x), 0), w.keys) for x in k_len) if k_len is not None else w.B * w.keys)
     return 2.0 * n_elem + 2 * 2.0 * kv_rows * w.d + 4.0 * n_elem + 4.0 * w.B * w.H * w.N
 
 
@@ -187,8 +187,9 @@ def dist_setup(args):
 
 def workload_config(w, world: int, q_bytes: int) -> dict:
     """The `config` object of the JSON line (identical for both arms)."""
-    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "N": w.N, "d": w.d,
-            "causal": w.causal, "out": "fp32 O + fp32 lse", "flops_per_step_per_gpu": w.flops(),
+    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "N": w.N, "N_k": w.keys, "d": w.d,
+            "causal": w.causal, "key_splits": w.splits, "out": "fp32 O + fp32 lse",
+            "flops_per_step_per_gpu": w.flops(),
             "l2": "inputs larger than L2 (Q,K,V %.0f MB > 126 MB); no flush" % (q_bytes / 1e6),
             "parallelism": f"replicas x{world}"}
 
@@ -215,9 +216,9 @@ def oracle_rows_flops(w, rows, k_len) -> float:
     for r in rows:
         bh, i = divmod(int(r), w.N)
         b = bh // w.H
-        e = w.N if k_len is None else max(0, min(w.N, int(k_len[b])))
+        e = w.keys if k_len is None else max(0, min(w.keys, int(k_len[b])))
         if w.causal:
-            e = min(e, i + 1)
+            e = min(e, max(0, i + 1 + w.keys - w.N))
         tot += e
     return 4.0 * w.d * tot
 
@@ -299,7 +300,11 @@ def run_ours(args, world, rank, local):
     o = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.float32, device=dev)
     lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    params = fb.make_params(qd, kd, vd, o, lse, w.causal, w.scale, k_len=kld)
+    splits = fb.suggest_splits(qd, kd) if w.splits < 0 else w.splits
+    ws = None
+    if splits > 1:
+        ws = torch.empty(max(fb.workspace_bytes(qd, kd, splits), 16), dtype=torch.uint8, device=dev)
+    params = fb.make_params(qd, kd, vd, o, lse, w.causal, w.scale, k_len=kld, num_splits=splits, workspace=ws)
     lib = fb.load()
     sptr = fb._stream(stream)
     import ctypes
@@ -353,14 +358,14 @@ def run_ours(args, world, rank, local):
         oh = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.float32).pin_memory()
         lh = torch.empty(w.B, w.H, w.N, dtype=torch.float32).pin_memory()
         fb.fa_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, w.causal, w.scale, k_len_h=klh, k_len_d=kld,
-                       stream=stream)
+                       stream=stream, num_splits=splits, workspace=ws)
         barrier(world)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.e2e_steps):
             fb.fa_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, w.causal, w.scale, k_len_h=klh,
-                           k_len_d=kld, stream=stream)
+                           k_len_d=kld, stream=stream, num_splits=splits, workspace=ws)
         e1.record(stream)
         e1.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
@@ -379,7 +384,9 @@ def run_ours(args, world, rank, local):
     traffic = measured_traffic(args.workload)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_src} bf16_tflops (burst)",
-                "kernel": "fa_fwd_sm100_kernel", "kernel_ms": kernel_ms,
+                "kernel": "fa_fwd_sm100_kernel" + (" + fa_combine_kernel (split pass and merge, one event pair)"
+                                                   if splits > 1 else ""),
+                "kernel_ms": kernel_ms,
                 "algorithmic_bytes": alg_bytes, "hbm_gbs_algorithmic": alg_bytes / (kernel_ms * 1e-3) / 1e9,
                 "hbm_peak_gbs": float(peaks["hbm_gbs"])}
     cpu = None
@@ -395,7 +402,7 @@ def run_ours(args, world, rank, local):
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (2 if splits > 1 else 1),
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

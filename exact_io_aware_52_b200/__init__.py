@@ -8,6 +8,6 @@ computes attention on the CPU: when the library is missing, calls fail loudly.
 from ._binding import (  # noqa: F401
     FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT, FA_ERR_INVALID_ARGUMENT, FA_ERR_MISALIGNED, FA_ERR_UNSUPPORTED,
     FA_FLAG_EAGER_RESCALE, FA_O_BF16, FA_O_F32, FA_OK, FaError, attention, fa_fwd, fa_fwd_ex, fa_fwd_host,
-    read_device_status, status_string, version,
+    read_device_status, status_string, suggest_splits, version, workspace_bytes,
 )
 from .workloads import WORKLOADS, Workload, make_inputs, sample_rows  # noqa: F401

@@ -39,6 +39,8 @@ class FaParams(ctypes.Structure):
         ("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int),
         ("causal", ctypes.c_int), ("scale", ctypes.c_float), ("o_dtype", ctypes.c_int),
         ("flags", ctypes.c_int), ("timeout_ms", ctypes.c_uint32), ("H_kv", ctypes.c_int),
+        ("N_k", ctypes.c_int), ("num_splits", ctypes.c_int), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
     ]
 
 
@@ -79,6 +81,10 @@ def load():
             lib.fa_status_string.argtypes = [i]
             lib.fa_version.restype = i
             lib.fa_version.argtypes = []
+            lib.fa_fwd_workspace_bytes.restype = ctypes.c_size_t
+            lib.fa_fwd_workspace_bytes.argtypes = [ctypes.POINTER(FaParams)]
+            lib.fa_fwd_suggest_splits.restype = i
+            lib.fa_fwd_suggest_splits.argtypes = [ctypes.POINTER(FaParams)]
             _lib = lib
     return _lib
 
@@ -141,33 +147,59 @@ def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
 
 
 def make_params(q, k, v, o, lse, causal, scale, k_len=None, dev_status=None, flags=0, timeout_ms=0,
-                shape=None) -> FaParams:
-    """Fill a fa_fwd_params from tensors (any of them may be None for argument tests)."""
+                shape=None, num_splits=0, workspace=None) -> FaParams:
+    """Fill a fa_fwd_params from tensors (any of them may be None for argument tests).
+
+    k, v may be [B, H_kv, N_k, d] with H_kv dividing H and any N_k; workspace is a
+    CUDA tensor of at least workspace_bytes(...) bytes when num_splits > 1."""
     import torch
     if shape is None:
         shape = tuple(q.shape)
     B, H, N, d = shape
     o_dtype = FA_O_BF16 if (o is not None and o.dtype == torch.bfloat16) else FA_O_F32
-    H_kv = int(k.shape[1]) if (k is not None and hasattr(k, "shape") and k.dim() == 4) else 0
+    kv4 = k is not None and hasattr(k, "shape") and k.dim() == 4
+    H_kv = int(k.shape[1]) if kv4 else 0
+    N_k = int(k.shape[2]) if kv4 else 0
+    if kv4 and N_k == 0 and B * H * N > 0:
+        # N_k = 0 means "N keys" in the C ABI; an empty key tensor is key padding (k_len = 0)
+        raise ValueError("k and v have no keys: pass at least one key row and k_len = 0")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     return FaParams(q=_ptr(q), k=_ptr(k), v=_ptr(v), o=_ptr(o), lse=_ptr(lse), k_len=_ptr(k_len),
                     dev_status=_ptr(dev_status), B=B, H=H, N=N, d=d, causal=int(bool(causal)),
                     scale=float(scale), o_dtype=o_dtype, flags=int(flags), timeout_ms=int(timeout_ms),
-                    H_kv=H_kv)
+                    H_kv=H_kv, N_k=N_k, num_splits=int(num_splits), workspace=_ptr(workspace),
+                    workspace_bytes=ws_bytes)
+
+
+def workspace_bytes(q, k, num_splits: int) -> int:
+    """Scratch bytes a num_splits > 1 call needs (fa_fwd_workspace_bytes)."""
+    p = make_params(q, k, None, None, None, False, 1.0, num_splits=num_splits)
+    return int(load().fa_fwd_workspace_bytes(ctypes.byref(p)))
+
+
+def suggest_splits(q, k) -> int:
+    """The library's key-split count for this shape on the current device."""
+    p = make_params(q, k, None, None, None, False, 1.0)
+    return int(load().fa_fwd_suggest_splits(ctypes.byref(p)))
 
 
 def fa_fwd_ex(q, k, v, o, lse, causal: bool, scale: float, k_len=None, dev_status=None, flags: int = 0,
-              timeout_ms: int = 0, stream=None):
+              timeout_ms: int = 0, stream=None, num_splits: int = 0, workspace=None):
     """fa_fwd_ex: as fa_fwd, plus k_len (int32 [B] CUDA tensor), o may be bf16,
     an optional int32 status word, FA_FLAG_* flags and the wait time limit.
-    k and v may have fewer heads than q ([B, H_kv, N, d], H_kv dividing H)."""
-    p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms)
+    k and v may be [B, H_kv, N_k, d] (grouped heads, more keys than queries);
+    num_splits > 1 splits each row's keys, with `workspace` as scratch."""
+    p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms,
+                    num_splits=num_splits, workspace=workspace)
     _check(load().fa_fwd_ex(ctypes.byref(p), _stream(stream)), "fa_fwd_ex")
 
 
 def fa_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal: bool, scale: float,
-                k_len_h=None, k_len_d=None, dev_status=None, flags: int = 0, stream=None):
+                k_len_h=None, k_len_d=None, dev_status=None, flags: int = 0, stream=None, num_splits: int = 0,
+                workspace=None):
     """fa_fwd_host: host (pinned) tensors in and out, device tensors as staging."""
-    dev = make_params(q_d, k_d, v_d, o_d, lse_d, causal, scale, k_len_d, dev_status, flags)
+    dev = make_params(q_d, k_d, v_d, o_d, lse_d, causal, scale, k_len_d, dev_status, flags,
+                      num_splits=num_splits, workspace=workspace)
     hp = FaHostParams(q=_ptr(q_h), k=_ptr(k_h), v=_ptr(v_h), k_len=_ptr(k_len_h), o=_ptr(o_h), lse=_ptr(lse_h),
                       dev=dev)
     _check(load().fa_fwd_host(ctypes.byref(hp), _stream(stream)), "fa_fwd_host")
@@ -177,14 +209,22 @@ def read_device_status(dev_status, stream=None) -> int:
     return load().fa_read_device_status(_ptr(dev_status), _stream(stream))
 
 
-def attention(q, k, v, causal: bool, scale: float, k_len=None, out_dtype=None, flags: int = 0, stream=None):
-    """Allocate O and lse with torch on q's device and run fa_fwd_ex.
+def attention(q, k, v, causal: bool, scale: float, k_len=None, out_dtype=None, flags: int = 0, stream=None,
+              num_splits: int = 0):
+    """Allocate O, lse (and any split workspace) with torch on q's device and run fa_fwd_ex.
 
+    num_splits: 0 = none, -1 = the library's suggestion, S > 1 = S key splits.
     Returns (O [B,H,N,d] in out_dtype (fp32 default), lse [B,H,N] fp32).
     """
     import torch
     B, H, N, d = q.shape
     o = torch.empty((B, H, N, d), dtype=out_dtype or torch.float32, device=q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    fa_fwd_ex(q, k, v, o, lse, causal, scale, k_len=k_len, flags=flags, stream=stream)
+    if num_splits < 0:
+        num_splits = suggest_splits(q, k)
+    ws = None
+    if num_splits > 1:
+        ws = torch.empty(max(workspace_bytes(q, k, num_splits), 16), dtype=torch.uint8, device=q.device)
+    fa_fwd_ex(q, k, v, o, lse, causal, scale, k_len=k_len, flags=flags, stream=stream, num_splits=num_splits,
+              workspace=ws)
     return o, lse

@@ -11,12 +11,14 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_combine_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0
 constexpr int kMaxDevices = 64;
+constexpr int kMaxSplits = 1024;
 
 struct DeviceInfo {
     bool probed = false;
@@ -88,6 +90,7 @@ fa_status validate(const fa_fwd_params *p) {
     if (p->o_dtype != FA_O_F32 && p->o_dtype != FA_O_BF16) return FA_ERR_INVALID_ARGUMENT;
     if (p->flags & ~FA_FLAG_EAGER_RESCALE) return FA_ERR_INVALID_ARGUMENT;
     if (p->H_kv < 0 || (p->H_kv > 0 && p->H % p->H_kv != 0)) return FA_ERR_INVALID_ARGUMENT;
+    if (p->N_k < 0 || p->num_splits < 0 || p->num_splits > kMaxSplits) return FA_ERR_INVALID_ARGUMENT;
     if (p->d != 64 && p->d != 128) return FA_ERR_UNSUPPORTED;
     const long long rows = (long long)p->B * p->H * p->N;
     if (rows == 0) return FA_OK;
@@ -98,7 +101,39 @@ fa_status validate(const fa_fwd_params *p) {
     if ((reinterpret_cast<uintptr_t>(p->lse) & 3u) || (reinterpret_cast<uintptr_t>(p->k_len) & 3u) ||
         (reinterpret_cast<uintptr_t>(p->dev_status) & 3u))
         return FA_ERR_MISALIGNED;
+    if (p->num_splits > 1) {
+        if (!p->workspace || p->workspace_bytes < fa_fwd_workspace_bytes(p)) return FA_ERR_INVALID_ARGUMENT;
+        if (!aligned16(p->workspace)) return FA_ERR_MISALIGNED;
+    }
     return FA_OK;
+}
+
+// Key tiles of 128 keys and the split layout actually used for *p.
+struct SplitPlan {
+    int n_k;          // keys
+    int splits;       // effective split count (no empty trailing splits)
+    int split_tiles;  // key tiles per split
+};
+
+SplitPlan plan_splits(const fa_fwd_params *p) {
+    SplitPlan sp;
+    sp.n_k = p->N_k > 0 ? p->N_k : p->N;
+    const int tiles = (sp.n_k + fa::BN - 1) / fa::BN;
+    int s = p->num_splits > 1 ? p->num_splits : 1;
+    if (s > tiles) s = tiles > 0 ? tiles : 1;
+    sp.split_tiles = tiles > 0 ? (tiles + s - 1) / s : 1;
+    sp.splits = tiles > 0 ? (tiles + sp.split_tiles - 1) / sp.split_tiles : 1;
+    return sp;
+}
+
+template <int D, bool BF16>
+fa_status launch_combine(const float *o_part, const float *lse_part, void *o, float *lse, int splits, long long rows,
+                         int num_sms, cudaStream_t stream) {
+    const long long warps = rows;
+    long long blocks = (warps * 32 + 255) / 256;
+    if (blocks > 8LL * num_sms) blocks = 8LL * num_sms;
+    fa::fa_combine_kernel<D, BF16><<<(int)blocks, 256, 0, stream>>>(o_part, lse_part, o, lse, splits, rows);
+    return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 template <int D, bool BF16>
@@ -140,20 +175,35 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     std::memset(&kp, 0, sizeof kp);
     const int BH = p->B * p->H;
     const int H_kv = p->H_kv > 0 ? p->H_kv : p->H;
+    const SplitPlan sp = plan_splits(p);
     if ((st = encode_map(&kp.tm_q, p->q, BH, p->N, p->d)) != FA_OK) return st;
-    if ((st = encode_map(&kp.tm_k, p->k, p->B * H_kv, p->N, p->d)) != FA_OK) return st;
-    if ((st = encode_map(&kp.tm_v, p->v, p->B * H_kv, p->N, p->d)) != FA_OK) return st;
-    kp.o = p->o;
-    kp.lse = p->lse;
+    // a map over zero keys is not encodable; with N_k = 0 no key tile is loaded
+    const int n_k_map = sp.n_k > 0 ? sp.n_k : 1;
+    if ((st = encode_map(&kp.tm_k, p->k, p->B * H_kv, n_k_map, p->d)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_v, p->v, p->B * H_kv, n_k_map, p->d)) != FA_OK) return st;
+    const long long rows = (long long)BH * p->N;
+    float *o_part = nullptr, *lse_part = nullptr;
+    if (sp.splits > 1) {  // partials: fp32 [S][rows][d], then fp32 [S][rows]
+        o_part = static_cast<float *>(p->workspace);
+        lse_part = o_part + (size_t)sp.splits * rows * p->d;
+        kp.o = o_part;
+        kp.lse = lse_part;
+    } else {
+        kp.o = p->o;
+        kp.lse = p->lse;
+    }
     kp.k_len = p->k_len;
     kp.status = p->dev_status;
     kp.B = p->B;
     kp.H = p->H;
+    kp.N = p->N;
+    kp.Nk = sp.n_k;
     kp.group = p->H / H_kv;
     kp.H_kv = H_kv;
-    kp.N = p->N;
     kp.n_blocks = (p->N + fa::kUnitRows - 1) / fa::kUnitRows;
-    kp.n_units = BH * kp.n_blocks;
+    kp.n_splits = sp.splits;
+    kp.split_tiles = sp.split_tiles;
+    kp.n_units = BH * kp.n_blocks * sp.splits;
     kp.causal = p->causal;
     kp.scale_log2 = (float)((double)p->scale * 1.4426950408889634074);
     kp.tau = (p->flags & FA_FLAG_EAGER_RESCALE) ? 0.f : 8.f;
@@ -162,8 +212,58 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     const int grid = kp.n_units < di->num_sms ? kp.n_units : di->num_sms;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = p->o_dtype == FA_O_BF16;
+    if (sp.splits > 1) {  // the split pass always writes fp32 partials; the merge writes the output type
+        st = (p->d == 64) ? launch<64, false>(kp, *di, grid, s) : launch<128, false>(kp, *di, grid, s);
+        if (st != FA_OK) return st;
+        if (p->d == 64)
+            return bf16 ? launch_combine<64, true>(o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)
+                        : launch_combine<64, false>(o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s);
+        return bf16 ? launch_combine<128, true>(o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)
+                    : launch_combine<128, false>(o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s);
+    }
     if (p->d == 64) return bf16 ? launch<64, true>(kp, *di, grid, s) : launch<64, false>(kp, *di, grid, s);
     return bf16 ? launch<128, true>(kp, *di, grid, s) : launch<128, false>(kp, *di, grid, s);
+}
+
+size_t fa_fwd_workspace_bytes(const fa_fwd_params *p) {
+    if (!p || p->num_splits <= 1 || p->B <= 0 || p->H <= 0 || p->N <= 0 || (p->d != 64 && p->d != 128)) return 0;
+    const SplitPlan sp = plan_splits(p);
+    if (sp.splits <= 1) return 0;
+    const size_t rows = (size_t)p->B * p->H * p->N;
+    return (size_t)sp.splits * rows * ((size_t)p->d + 1) * sizeof(float);
+}
+
+int fa_fwd_suggest_splits(const fa_fwd_params *p) {
+    if (!p || p->B <= 0 || p->H <= 0 || p->N <= 0) return 0;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return 0;
+    const long long units = (long long)p->B * p->H * ((p->N + fa::kUnitRows - 1) / fa::kUnitRows);
+    const long long n_k = p->N_k > 0 ? p->N_k : p->N;
+    const long long tiles = (n_k + fa::BN - 1) / fa::BN;
+    if (units >= 2LL * sms || tiles <= 1) return 1;
+    // Cost model in key-tile steps of one persistent CTA: waves of units times the
+    // tiles of the longest split plus a fixed per-unit cost (Q load, drain,
+    // epilogue ~ 2 steps), plus the partials' write and re-read (8 (d + 1) bytes
+    // per row and split) at ~16 MB of HBM traffic per step across the GPU.
+    const double rows = (double)p->B * p->H * p->N;
+    const double split_cost = rows * 8.0 * (p->d + 1) / 16.0e6;
+    long long best_s = 1;
+    double best = 0.0;
+    const long long s_max = tiles < kMaxSplits ? tiles : kMaxSplits;
+    for (long long s = 1; s <= s_max; ++s) {
+        const long long per = (tiles + s - 1) / s;
+        const long long eff = (tiles + per - 1) / per;  // splits left after dropping empty ones
+        if (eff != s) continue;
+        const long long waves = (units * s + sms - 1) / sms;
+        const double cost = (double)waves * (double)(per + 2) + (s > 1 ? split_cost * (double)s : 0.0);
+        if (s == 1 || cost < best) {
+            best = cost;
+            best_s = s;
+        }
+    }
+    return (int)best_s;
 }
 
 fa_status fa_fwd(const void *q, const void *k, const void *v, float *o, float *lse, int B, int H, int N, int d,
@@ -196,7 +296,8 @@ fa_status fa_fwd_host(const fa_fwd_host_params *hp, void *stream) {
     if ((hp->k_len == nullptr) != (p->k_len == nullptr)) return FA_ERR_INVALID_ARGUMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t q_bytes = rows * p->d * 2;
-    const size_t kv_bytes = (size_t)p->B * (p->H_kv > 0 ? p->H_kv : p->H) * p->N * p->d * 2;
+    const size_t kv_bytes =
+        (size_t)p->B * (p->H_kv > 0 ? p->H_kv : p->H) * (p->N_k > 0 ? p->N_k : p->N) * p->d * 2;
     const size_t o_bytes = rows * p->d * (p->o_dtype == FA_O_BF16 ? 2 : 4);
     if (cudaMemcpyAsync(const_cast<void *>(p->q), hp->q, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(const_cast<void *>(p->k), hp->k, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||

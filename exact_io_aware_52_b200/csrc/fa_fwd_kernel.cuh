@@ -82,17 +82,20 @@ __device__ __forceinline__ uint32_t col_s(uint32_t x) { return x * 128u; }      
 __device__ __forceinline__ uint32_t col_o(uint32_t x, uint32_t d) { return 256u + x * d; }  // O_X
 
 struct FwdParams {
-    CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps over [B*H][N][D] (Q) and [B*H_kv][N][D] (K, V) bf16;
+    CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps over [B*H][N][D] (Q) and [B*H_kv][Nk][D] (K, V) bf16;
                                    // box {64, 128, 1}; 128-byte swizzle
-    void *o;                       // [B, H, N, D] fp32 or bf16
-    float *lse;                    // [B, H, N]
+    void *o;                       // [n_splits][B, H, N, D] fp32 or bf16 (n_splits > 1: fp32 partials)
+    float *lse;                    // [n_splits][B, H, N]
     const int32_t *k_len;          // [B] or nullptr
     int32_t *status;               // device status word or nullptr
-    int B, H, N;
+    int B, H, N;                   // N queries
+    int Nk;                        // keys; query i sits at key position i + Nk - N
     int H_kv;                      // key/value heads; query head h uses key/value head h / group
     int group;                     // H / H_kv
     int n_blocks;                  // ceil(N / 256)
-    int n_units;                   // B * H * n_blocks
+    int n_splits;                  // key-range splits per query block (1: none)
+    int split_tiles;               // key tiles per split
+    int n_units;                   // B * H * n_blocks * n_splits
     int causal;
     float scale_log2;              // scale * log2(e)
     float tau;                     // rescale threshold in log2 units (<= 0: rescale on any growth)
@@ -133,9 +136,10 @@ struct Cfg {
 };
 
 struct UnitCoord {
-    int bh, b, blk;
+    int bh, b, blk, split;
     int bh_kv;  // key/value head row of K and V: b * H_kv + h / group
-    int n[2];  // key tiles of query tile A and B (a prefix [0, n) of the key tiles)
+    int lo;     // first key tile of this unit's key range
+    int n[2];   // key tiles of query tile A and B: tiles [lo, lo + n[x])
     int nmax;
 };
 
@@ -148,21 +152,27 @@ __device__ __forceinline__ int unit_index(int k) {
 }
 
 // Units are numbered head-major (the CTAs working at one time share a few
-// heads' K and V in L2), longest (causal) query blocks first within a head.
+// heads' K and V in L2), longest (causal) query blocks first within a head,
+// key splits innermost.  Query tile x of the unit covers the key tiles of the
+// unit's split that some row of the tile may attend to.
 __device__ __forceinline__ UnitCoord decode_unit(const FwdParams &p, int t) {
     UnitCoord u;
-    u.blk = p.n_blocks - 1 - t % p.n_blocks;
-    u.bh = t / p.n_blocks;
+    u.split = t % p.n_splits;
+    const int r = t / p.n_splits;
+    u.blk = p.n_blocks - 1 - r % p.n_blocks;
+    u.bh = r / p.n_blocks;
     u.b = u.bh / p.H;
     u.bh_kv = u.b * p.H_kv + (u.bh - u.b * p.H) / p.group;
-    int kv_lim = p.N;
-    if (p.k_len) kv_lim = min(max(__ldg(p.k_len + u.b), 0), p.N);
+    u.lo = u.split * p.split_tiles;
+    int kv_lim = p.Nk;
+    if (p.k_len) kv_lim = min(max(__ldg(p.k_len + u.b), 0), p.Nk);
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
         const int first = u.blk * kUnitRows + x * BM;
-        int e = kv_lim;
-        if (p.causal) e = min(e, first + BM);
-        u.n[x] = (first < p.N) ? (e + BN - 1) / BN : 0;
+        int e = kv_lim;  // keys [0, e) may be attended to by some row of the tile
+        if (p.causal) e = max(0, min(e, first + BM + (p.Nk - p.N)));
+        const int tiles = (first < p.N) ? (e + BN - 1) / BN : 0;
+        u.n[x] = max(0, min(tiles, u.lo + p.split_tiles) - u.lo);
     }
     u.nmax = max(u.n[0], u.n[1]);
     return u;
@@ -297,15 +307,16 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         const UnitCoord u = decode_unit(p, t);
         const int row = u.blk * kUnitRows + x * BM + row_in_tile;
         const bool row_valid = row < p.N;
-        const size_t row_id = (size_t)u.bh * p.N + row;
+        // output row: [split][B*H][N] (the split index is 0 without key splits)
+        const size_t row_id = ((size_t)u.split * p.B * p.H + u.bh) * p.N + row;
         const int n = u.n[x];
         if (n == 0) {  // no allowed key for these rows: O = 0, lse = -inf
             if (row_valid) fill_row<D, O_BF16>(p.o, p.lse, row_id, false, NEG_INF);
             continue;
         }
-        int lim = p.N;
-        if (p.k_len) lim = min(max(__ldg(p.k_len + u.b), 0), p.N);
-        if (p.causal) lim = min(lim, row + 1);
+        int lim = p.Nk;  // keys [0, lim) are allowed for this row
+        if (p.k_len) lim = min(max(__ldg(p.k_len + u.b), 0), p.Nk);
+        if (p.causal) lim = min(lim, row + 1 + (p.Nk - p.N));
 
         float m_ref = 0.f;  // reference maximum, log2 units
         float l = 0.f;      // running sum of 2^(x - m_ref), unrounded: gives lse
@@ -318,7 +329,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             if (!ok) break;
             tc_fence_after();
 
-            const int kv0 = j * BN;
+            const int kv0 = (u.lo + j) * BN;
             const bool masked = kv0 + BN > lim;  // masking step: keys at or beyond the row's limit
             float s[BN];
             uint32_t pk0[32], pk1[32];          // P for keys [0,64) and [64,128), two bf16 per column
@@ -383,7 +394,10 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             break;
         }
         tc_fence_after();
-        const float inv_l = 1.f / lr;
+        // a row whose allowed keys all lie outside this unit's key range (key
+        // splits) has nothing summed: O = 0, lse = -inf for it
+        const bool empty = !(lr > 0.f);
+        const float inv_l = empty ? 0.f : 1.f / lr;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
             uint32_t r[32];
@@ -392,7 +406,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             tmem_reg_fence(r);
             if (row_valid) store_row_chunk<D, O_BF16>(p.o, row_id, ch, r, inv_l);
         }
-        if (row_valid) p.lse[row_id] = (m_ref + log2f(l)) * LN2;
+        if (row_valid) p.lse[row_id] = empty ? NEG_INF : (m_ref + log2f(l)) * LN2;
         tc_fence_before();
         mbar_arrive(o_free);
         ++tl;
@@ -520,7 +534,7 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_3d(sK + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_k, &bars[C::kBarKFull + slot],
-                                c * 64, j * BN, u.bh_kv);
+                                c * 64, (u.lo + j) * BN, u.bh_kv);
                 ++gk;
             }
             {
@@ -533,7 +547,7 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_3d(sV + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_v, &bars[C::kBarVFull + slot],
-                                c * 64, j * BN, u.bh_kv);
+                                c * 64, (u.lo + j) * BN, u.bh_kv);
                 ++gv;
             }
         }

@@ -32,6 +32,8 @@ class Workload:
     kpad: tuple | None = None          # (lo, hi) inclusive range of key lengths, or None
     sample_rows_per_head: int | None = None  # rows the oracle checks per head (None: all)
     H_kv: int | None = None            # key/value heads (grouped attention); None: H
+    Nk: int | None = None              # keys (more keys than queries: cached keys); None: N
+    splits: int = 0                    # key splits the benchmark uses (0: none, -1: library's choice)
     seed: int = 0
     notes: str = field(default="", compare=False)
 
@@ -44,10 +46,19 @@ class Workload:
     def kv_heads(self) -> int:
         return self.H if self.H_kv is None else self.H_kv
 
+    @property
+    def keys(self) -> int:
+        return self.N if self.Nk is None else self.Nk
+
     def flops(self) -> float:
-        """Nominal attention FLOPs: 4*B*H*N^2*d, halved when causal."""
-        f = 4.0 * self.B * self.H * self.N * self.N * self.d
-        return f / 2 if self.causal else f
+        """Nominal attention FLOPs: 4*B*H*N^2*d, halved when causal; with N_k != N,
+        4*B*H*d times the allowed (query, key) pairs (bottom-right causal mask)."""
+        if self.Nk is None or self.Nk == self.N:
+            f = 4.0 * self.B * self.H * self.N * self.N * self.d
+            return f / 2 if self.causal else f
+        N, Nk = self.N, self.Nk
+        pairs = sum(max(0, min(Nk, i + 1 + Nk - N)) for i in range(N)) if self.causal else N * Nk
+        return 4.0 * self.B * self.H * self.d * pairs
 
 
 # The five workloads; seeds are 52000 + workload number.
@@ -63,19 +74,22 @@ WORKLOADS = {
     # grouped key/value heads (multi-query family): 8 key/value heads serve 32 query heads
     6: Workload("long-context causal grouped-KV B1 H32 Hkv8 N16384 d128", 1, 32, 16384, 128, True,
                 sample_rows_per_head=128, seed=52006, H_kv=8),
+    # cached keys: 256 new queries per head against 128K keys, key range split across SMs
+    7: Workload("cached-keys causal grouped-KV B1 H32 Hkv8 Nq256 Nk131072 d128 split-KV", 1, 32, 256, 128, True,
+                sample_rows_per_head=16, seed=52007, H_kv=8, Nk=131072, splits=-1),
 }
 
 
 def make_inputs(w: Workload, seed: int | None = None):
     """Draw (q, k, v, k_len) on the CPU for workload ``w``.
 
-    q: bfloat16 [B, H, N, d]; k, v: bfloat16 [B, H_kv, N, d] contiguous CPU tensors.
+    q: bfloat16 [B, H, N, d]; k, v: bfloat16 [B, H_kv, N_k, d] contiguous CPU tensors.
     k_len: int32 [B] CPU tensor, or None when the workload has no key padding.
     """
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed if seed is None else seed)
     shape = (w.B, w.H, w.N, w.d)
-    kv_shape = (w.B, w.kv_heads, w.N, w.d)
+    kv_shape = (w.B, w.kv_heads, w.keys, w.d)
     q = (torch.randn(shape, generator=g, dtype=torch.float32) * w.qk_std).to(torch.bfloat16)
     k = (torch.randn(kv_shape, generator=g, dtype=torch.float32) * w.qk_std).to(torch.bfloat16)
     v = torch.randn(kv_shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
@@ -107,6 +121,8 @@ def sample_rows(w: Workload, seed: int | None = None):
     return np.concatenate(out)
 
 
-def custom(B, H, N, d, causal, qk_std=1.0, kpad=None, seed=1, name="custom", H_kv=None) -> Workload:
+def custom(B, H, N, d, causal, qk_std=1.0, kpad=None, seed=1, name="custom", H_kv=None, Nk=None,
+           splits=0) -> Workload:
     """A workload of arbitrary shape (tests of ragged and edge shapes)."""
-    return Workload(name, B, H, N, d, causal, qk_std=qk_std, kpad=kpad, seed=seed, H_kv=H_kv)
+    return Workload(name, B, H, N, d, causal, qk_std=qk_std, kpad=kpad, seed=seed, H_kv=H_kv, Nk=Nk,
+                    splits=splits)

@@ -16,15 +16,18 @@
  *
  * Layout (all tensors contiguous, row-major):
  *   q       : bf16  [B, H, N, d]      (one N x d matrix per (b, h))
- *   k, v    : bf16  [B, H_kv, N, d]   (fa_fwd: H_kv = H; fa_fwd_ex may group:
- *             query head h attends with key/value head h / (H / H_kv), the
- *             multi-query attention of section "FlashAttention-2 (2023)")
+ *   k, v    : bf16  [B, H_kv, N_k, d] (fa_fwd: H_kv = H and N_k = N; fa_fwd_ex
+ *             may group heads -- query head h attends with key/value head
+ *             h / (H / H_kv), the multi-query attention of section
+ *             "FlashAttention-2 (2023)" -- and may give more keys than queries,
+ *             the cached-keys setting of section "Soluciones especializadas":
+ *             query i then sits at key position i + N_k - N)
  *   o       : fp32  [B, H, N, d]  (fa_fwd; fa_fwd_ex may select bf16)
  *   lse     : fp32  [B, H, N]
  *   k_len   : int32 [B]  (fa_fwd_ex only; key j of batch b is masked iff
  *             j >= k_len[b]; values are clamped to [0, N] on the device)
- * Mask: causal masks key j for query i when j > i (queries and keys share
- * positions 0..N-1).  A row with no allowed key gets O = 0, lse = -inf.
+ * Mask: causal masks key j for query i when j > i + N_k - N (j > i when
+ * N_k = N).  A row with no allowed key gets O = 0, lse = -inf.
  *
  * Ownership: the caller owns every buffer.  The library allocates, frees and
  * synchronises nothing (except fa_read_device_status and fa_fwd_host, which
@@ -39,6 +42,7 @@
 #ifndef EXACT_IO_AWARE_52_FA_H
 #define EXACT_IO_AWARE_52_FA_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -101,9 +105,38 @@ typedef struct {
     int o_dtype;             /* fa_o_dtype                                            */
     int flags;               /* FA_FLAG_* bits, 0 by default                          */
     uint32_t timeout_ms;     /* per-wait time limit on the device; 0 = 2000 ms        */
-    int H_kv;                /* key/value heads (k, v are [B, H_kv, N, d]); 0 means H;
+    int H_kv;                /* key/value heads (k, v are [B, H_kv, N_k, d]); 0 means H;
                                 must divide H (1 = multi-query attention)             */
+    int N_k;                 /* keys; 0 means N (queries); query i sits at key
+                                position i + N_k - N                                  */
+    int num_splits;          /* 0 or 1: one pass over each row's keys.  S > 1: the key
+                                range is cut into S contiguous parts processed in
+                                parallel (more work units when B*H*ceil(N/256) is
+                                below the SM count), their partial results written
+                                to `workspace` and merged by a second kernel          */
+    void *workspace;         /* device scratch, 16-byte aligned, at least
+                                fa_fwd_workspace_bytes(p) bytes; unused when
+                                num_splits <= 1.  Owned by the caller; the library
+                                writes every byte it reads from it in the same call   */
+    size_t workspace_bytes;  /* size of workspace                                     */
 } fa_fwd_params;
+
+/*
+ * fa_fwd_workspace_bytes -- device scratch bytes fa_fwd_ex needs for *p
+ * (0 when p->num_splits <= 1): the partial outputs of the key splits, fp32
+ * [S][B, H, N, d] and [S][B, H, N].  Host arithmetic only; 0 for a NULL p.
+ */
+FA_EXPORT size_t fa_fwd_workspace_bytes(const fa_fwd_params *p);
+
+/*
+ * fa_fwd_suggest_splits -- a key-split count for *p on the current device.
+ * Returns 1 when the unsplit grid already gives every SM two work units or
+ * the keys fit one 128-key tile; otherwise the count in [1, key tiles] that
+ * minimises a cost model of whole waves of (query block, split) units over
+ * the SMs plus the partials' HBM round trip.  Returns 0 on error (NULL, a
+ * non-positive size, no CUDA device).
+ */
+FA_EXPORT int fa_fwd_suggest_splits(const fa_fwd_params *p);
 
 /*
  * fa_fwd_ex -- the forward pass with key padding, output dtype and a status

@@ -15,10 +15,11 @@ TOL_MEAN = 1e-3   # mean |O_gpu - O_ref|
 TOL_LSE = 1e-4    # max |lse_gpu - lse_ref| / max(|lse_ref|, 1)
 
 
-def run_gpu(q, k, v, causal, scale, k_len=None, out_dtype=torch.float32, flags=0, stream=None):
+def run_gpu(q, k, v, causal, scale, k_len=None, out_dtype=torch.float32, flags=0, stream=None, num_splits=0):
     """Run fa_fwd_ex on cuda:0; returns (O [B,H,N,d] fp32 CPU, lse [B,H,N] CPU).
 
-    Outputs start as NaN so rows the kernel fails to write are caught."""
+    Outputs (and any split workspace) start as NaN so rows the kernels fail to
+    write are caught.  num_splits = -1 takes the library's suggestion."""
     dev = torch.device("cuda:0")
     B, H, N, d = q.shape
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
@@ -26,7 +27,14 @@ def run_gpu(q, k, v, causal, scale, k_len=None, out_dtype=torch.float32, flags=0
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     o = torch.full((B, H, N, d), float("nan"), dtype=out_dtype, device=dev)
     lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
-    fb.fa_fwd_ex(qd, kd, vd, o, lse, causal, scale, k_len=kl, dev_status=status, flags=flags, stream=stream)
+    if num_splits < 0:
+        num_splits = fb.suggest_splits(qd, kd)
+    ws = None
+    if num_splits > 1:
+        nbytes = fb.workspace_bytes(qd, kd, num_splits)
+        ws = torch.full((max(nbytes, 16) // 4,), float("nan"), dtype=torch.float32, device=dev)
+    fb.fa_fwd_ex(qd, kd, vd, o, lse, causal, scale, k_len=kl, dev_status=status, flags=flags, stream=stream,
+                 num_splits=num_splits, workspace=ws)
     st = fb.read_device_status(status, stream=stream)
     assert st == fb.FA_OK, fb.status_string(st)
     return o.float().cpu(), lse.cpu()
@@ -51,8 +59,9 @@ def compare(o_rows, lse_rows, o_ref, lse_ref, tol_max=TOL_MAX, tol_mean=TOL_MEAN
     return stats
 
 
-def check_case(q, k, v, causal, scale, k_len=None, rows=None, out_dtype=torch.float32, flags=0, **tol):
-    o, lse = run_gpu(q, k, v, causal, scale, k_len=k_len, out_dtype=out_dtype, flags=flags)
+def check_case(q, k, v, causal, scale, k_len=None, rows=None, out_dtype=torch.float32, flags=0, num_splits=0,
+               **tol):
+    o, lse = run_gpu(q, k, v, causal, scale, k_len=k_len, out_dtype=out_dtype, flags=flags, num_splits=num_splits)
     B, H, N, d = q.shape
     o_ref, lse_ref = oracle.attention_f64(q, k, v, causal, scale, k_len=None if k_len is None else list(k_len),
                                           rows=rows)
@@ -66,5 +75,6 @@ def check_case(q, k, v, causal, scale, k_len=None, rows=None, out_dtype=torch.fl
 def check_workload(w: workloads.Workload, **kw):
     q, k, v, k_len = workloads.make_inputs(w)
     rows = None if w.sample_rows_per_head is None else workloads.sample_rows(w)
+    kw.setdefault("num_splits", w.splits)
     return check_case(q, k, v, w.causal, w.scale, k_len=None if k_len is None else k_len.tolist(),
                       rows=rows, **kw)

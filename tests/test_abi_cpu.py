@@ -43,12 +43,13 @@ def test_status_strings_and_version():
     for code, name in names.items():
         assert fb.status_string(code) == name
     assert fb.status_string(99) == "FA_ERR_UNKNOWN"
-    assert fb.version() == 100
+    assert fb.version() == 200
 
 
 def _params(**kw):
     base = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0x50000, k_len=None, dev_status=None,
-                B=1, H=2, N=128, d=64, causal=0, scale=0.125, o_dtype=0, flags=0, timeout_ms=0, H_kv=0)
+                B=1, H=2, N=128, d=64, causal=0, scale=0.125, o_dtype=0, flags=0, timeout_ms=0, H_kv=0,
+                N_k=0, num_splits=0, workspace=None, workspace_bytes=0)
     base.update(kw)
     return fb.FaParams(**base)
 
@@ -77,6 +78,12 @@ def _ex(**kw):
     (dict(H_kv=-1), fb.FA_ERR_INVALID_ARGUMENT),
     (dict(H=6, H_kv=4), fb.FA_ERR_INVALID_ARGUMENT),
     (dict(H=6, H_kv=7), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(N_k=-1), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(num_splits=-2), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(num_splits=5000), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(N_k=1024, num_splits=4), fb.FA_ERR_INVALID_ARGUMENT),              # no workspace
+    (dict(N_k=1024, num_splits=4, workspace=0x80000, workspace_bytes=64), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(N_k=1024, num_splits=4, workspace=0x80008, workspace_bytes=1 << 30), fb.FA_ERR_MISALIGNED),
     (dict(d=32), fb.FA_ERR_UNSUPPORTED),
     (dict(d=256), fb.FA_ERR_UNSUPPORTED),
     (dict(d=96), fb.FA_ERR_UNSUPPORTED),
@@ -95,6 +102,18 @@ def _ex(**kw):
 def test_argument_errors_are_synchronous(kw, expect):
     # none of these reaches the device: the pointers are never dereferenced
     assert _ex(**kw) == expect
+
+
+def test_workspace_bytes():
+    lib = fb.load()
+    p = _params(N_k=1000, num_splits=4)        # 8 key tiles -> 4 splits of 2 tiles
+    assert lib.fa_fwd_workspace_bytes(ctypes.byref(p)) == 4 * (1 * 2 * 128) * (64 + 1) * 4
+    p = _params(N_k=1000, num_splits=5)        # 5 requested -> 4 non-empty splits of 2 tiles
+    assert lib.fa_fwd_workspace_bytes(ctypes.byref(p)) == 4 * (1 * 2 * 128) * (64 + 1) * 4
+    p = _params(N_k=100, num_splits=8)         # one key tile: no split
+    assert lib.fa_fwd_workspace_bytes(ctypes.byref(p)) == 0
+    assert lib.fa_fwd_workspace_bytes(ctypes.byref(_params())) == 0
+    assert lib.fa_fwd_workspace_bytes(None) == 0
 
 
 def test_fa_fwd_validates_like_ex():

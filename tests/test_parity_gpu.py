@@ -25,7 +25,7 @@ def rand_inputs(B, H, N, d, seed, std=1.0):
 
 
 # ------------------------------------------------------------ the five workloads
-@pytest.mark.parametrize("wid", [1, 2, 3, 4, 5, 6])
+@pytest.mark.parametrize("wid", [1, 2, 3, 4, 5, 6, 7])
 def test_workload_parity(wid):
     """Each seeded workload at its full size, in the launch configuration the
     benchmark times (all rows for 1-3, the seeded row sample for 4-5)."""

@@ -21,6 +21,8 @@ FA_ERR_MISALIGNED = 2
 FA_ERR_UNSUPPORTED = 3
 FA_ERR_CUDA = 4
 FA_ERR_DEVICE_TIMEOUT = 5
+FA_ERR_WORKSPACE_LIMIT = 6
+FA_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024   # include/fa.h
 FA_O_F32 = 0
 FA_O_BF16 = 1
 FA_FLAG_EAGER_RESCALE = 1
@@ -85,6 +87,8 @@ def load():
             lib.fa_fwd_workspace_bytes.argtypes = [ctypes.POINTER(FaParams)]
             lib.fa_fwd_suggest_splits.restype = i
             lib.fa_fwd_suggest_splits.argtypes = [ctypes.POINTER(FaParams)]
+            lib.fa_fwd_static_workspace.restype = i
+            lib.fa_fwd_static_workspace.argtypes = [ctypes.POINTER(FaParams), ctypes.c_void_p]
             _lib = lib
     return _lib
 
@@ -192,6 +196,15 @@ def fa_fwd_ex(q, k, v, o, lse, causal: bool, scale: float, k_len=None, dev_statu
     p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms,
                     num_splits=num_splits, workspace=workspace)
     _check(load().fa_fwd_ex(ctypes.byref(p), _stream(stream)), "fa_fwd_ex")
+
+
+def fa_fwd_static_workspace(q, k, v, o, lse, causal: bool, scale: float, k_len=None, dev_status=None,
+                            flags: int = 0, timeout_ms: int = 0, stream=None, num_splits: int = 0):
+    """fa_fwd_static_workspace: fa_fwd_ex with the split scratch in the library's
+    fixed device array (FA_STATIC_WORKSPACE_BYTES per device, shared by all calls
+    on the device: do not overlap calls).  Allocates nothing."""
+    p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms, num_splits=num_splits)
+    _check(load().fa_fwd_static_workspace(ctypes.byref(p), _stream(stream)), "fa_fwd_static_workspace")
 
 
 def fa_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal: bool, scale: float,

@@ -16,10 +16,10 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libfa_sm100.so")
 SELFTEST_LIB = os.path.join(HERE, "libfa_selftest.so")
-# library -> its translation unit
+# library -> its translation units
 TARGETS = {
-    LIB: os.path.join(CSRC, "fa_api.cu"),
-    SELFTEST_LIB: os.path.join(CSRC, "selftest.cu"),
+    LIB: [os.path.join(CSRC, "fa_api.cu"), os.path.join(CSRC, "fa_static_workspace.cu")],
+    SELFTEST_LIB: [os.path.join(CSRC, "selftest.cu")],
 }
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + \
     [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
@@ -37,13 +37,13 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def _build_one(lib: str, src: str, force: bool, verbose: bool) -> str:
+def _build_one(lib: str, srcs: list, force: bool, verbose: bool) -> str:
     if not force and os.path.exists(lib):
         t = os.path.getmtime(lib)
-        if all(os.path.getmtime(f) <= t for f in [src, *HEADERS]):
+        if all(os.path.getmtime(f) <= t for f in [*srcs, *HEADERS]):
             return lib
     tmp = lib + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-shared", "-I", INCLUDE, "-I", CSRC, src, "-o", tmp, "-lcudart"]
+    cmd = [nvcc(), *NVCC_FLAGS, "-shared", "-I", INCLUDE, "-I", CSRC, *srcs, "-o", tmp, "-lcudart"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
@@ -54,7 +54,7 @@ def _build_one(lib: str, src: str, force: bool, verbose: bool) -> str:
 
 def build(force: bool = False, verbose: bool = False) -> list:
     """Compile every library that is older than its sources; returns their paths."""
-    return [_build_one(lib, src, force, verbose) for lib, src in TARGETS.items()]
+    return [_build_one(lib, srcs, force, verbose) for lib, srcs in TARGETS.items()]
 
 
 if __name__ == "__main__":

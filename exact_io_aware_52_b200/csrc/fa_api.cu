@@ -333,6 +333,7 @@ const char *fa_status_string(fa_status s) {
         case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
         case FA_ERR_CUDA: return "FA_ERR_CUDA";
         case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+        case FA_ERR_WORKSPACE_LIMIT: return "FA_ERR_WORKSPACE_LIMIT";
     }
     return "FA_ERR_UNKNOWN";
 }

@@ -61,7 +61,9 @@ typedef enum {
     FA_ERR_MISALIGNED = 2,       /* a pointer not 16-byte aligned (TMA requirement)   */
     FA_ERR_UNSUPPORTED = 3,      /* d not in {64, 128}, or the device is not sm_100    */
     FA_ERR_CUDA = 4,             /* a CUDA runtime/driver call or the launch failed   */
-    FA_ERR_DEVICE_TIMEOUT = 5    /* (device status word) a pipeline wait timed out     */
+    FA_ERR_DEVICE_TIMEOUT = 5,   /* (device status word) a pipeline wait timed out     */
+    FA_ERR_WORKSPACE_LIMIT = 6   /* fa_fwd_static_workspace: the splits need more than
+                                    FA_STATIC_WORKSPACE_BYTES of scratch                */
 } fa_status;
 
 typedef enum { FA_O_F32 = 0, FA_O_BF16 = 1 } fa_o_dtype;
@@ -175,6 +177,35 @@ FA_EXPORT const char *fa_status_string(fa_status s);
 
 /* Library version as an integer MAJOR*10000 + MINOR*100 + PATCH. */
 FA_EXPORT int fa_version(void);
+
+/* Size of the library's fixed device scratch array (64 MiB), per device. */
+#define FA_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
+
+/*
+ * fa_fwd_static_workspace -- fa_fwd_ex with the key-split scratch taken from
+ * a fixed device array inside the library instead of p->workspace, so that
+ * the call allocates no memory.  The pages have no counterpart: their
+ * forward pass has no key splits and hence no scratch; this is an interface
+ * convenience of this library.
+ *
+ * p is read as by fa_fwd_ex except that p->workspace and p->workspace_bytes
+ * are ignored.  With p->num_splits > 1 the scratch is a file-scope device
+ * array of FA_STATIC_WORKSPACE_BYTES; a problem whose splits need more
+ * (fa_fwd_workspace_bytes(p) > FA_STATIC_WORKSPACE_BYTES) is rejected with
+ * FA_ERR_WORKSPACE_LIMIT before anything is launched.  With num_splits <= 1
+ * no scratch is used and the call is fa_fwd_ex.
+ *
+ * The array is one per device and every call on that device uses it:
+ * calls whose executions overlap (on different streams, or from different
+ * host threads) race on it and their results are undefined.  Serialise them,
+ * e.g. on one stream.  Nothing in it has to start at zero.
+ *
+ * The first call with num_splits > 1 on a device looks the array's address
+ * up (cudaGetSymbolAddress, with that device current) and caches it; make
+ * that first call before any stream capture.  Errors: those of fa_fwd_ex,
+ * FA_ERR_WORKSPACE_LIMIT, and FA_ERR_CUDA if the lookup fails.
+ */
+FA_EXPORT fa_status fa_fwd_static_workspace(const fa_fwd_params *p, void *stream);
 
 #ifdef __cplusplus
 }

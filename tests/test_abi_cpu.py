@@ -39,7 +39,7 @@ def test_hidden_internals():
 
 def test_status_strings_and_version():
     names = {0: "FA_OK", 1: "FA_ERR_INVALID_ARGUMENT", 2: "FA_ERR_MISALIGNED", 3: "FA_ERR_UNSUPPORTED",
-             4: "FA_ERR_CUDA", 5: "FA_ERR_DEVICE_TIMEOUT"}
+             4: "FA_ERR_CUDA", 5: "FA_ERR_DEVICE_TIMEOUT", 6: "FA_ERR_WORKSPACE_LIMIT"}
     for code, name in names.items():
         assert fb.status_string(code) == name
     assert fb.status_string(99) == "FA_ERR_UNKNOWN"
@@ -124,6 +124,19 @@ def test_fa_fwd_validates_like_ex():
     assert lib.fa_fwd(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 1, 1, 128, 80, 0, f(0.125), None) == \
         fb.FA_ERR_UNSUPPORTED
     assert lib.fa_fwd(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 1, 1, 0, 64, 1, f(0.125), None) == fb.FA_OK
+
+
+def test_static_workspace_entry_validates():
+    lib = fb.load()
+    assert lib.fa_fwd_static_workspace(None, None) == fb.FA_ERR_INVALID_ARGUMENT
+    # splits needing more than the fixed array: rejected before any CUDA call
+    p = _params(H=8, N=1024, d=128, N_k=4096, num_splits=16)
+    assert lib.fa_fwd_workspace_bytes(ctypes.byref(p)) > fb.FA_STATIC_WORKSPACE_BYTES
+    assert lib.fa_fwd_static_workspace(ctypes.byref(p), None) == fb.FA_ERR_WORKSPACE_LIMIT
+    # without splits it is fa_fwd_ex: the same synchronous argument errors
+    assert lib.fa_fwd_static_workspace(ctypes.byref(_params(d=32)), None) == fb.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_static_workspace(ctypes.byref(_params(q=None)), None) == fb.FA_ERR_INVALID_ARGUMENT
+    assert lib.fa_fwd_static_workspace(ctypes.byref(_params(N=0)), None) == fb.FA_OK
 
 
 def test_host_entry_validates():

@@ -42,7 +42,7 @@ from exact_io_aware_52_b200 import workloads  # noqa: E402
 DEFAULT_WORKLOAD = 4  # long-context causal B1 H32 N16384 d128: the tensor-bound headline
 METRIC = "attention fwd TFLOP/s (bf16, 1xB200) and % of dense BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["fa_fwd_kernel.cuh", "sm100_ptx.cuh", "fa_api.cu"]
+KERNEL_SOURCES = ["fa_fwd_kernel.cuh", "sm100_ptx.cuh"]  # device code of the d <= 128 kernel (default record)
 
 
 def parse():
@@ -66,33 +66,37 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in (sources or KERNEL_SOURCES):
         with open(os.path.join(ROOT, "exact_io_aware_52_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def measured_traffic(workload_id: int):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "fa_fwd_traffic.txt")
-    if not os.path.exists(path):
-        return None
-    rec = {}
-    with open(path) as f:
-        for line in f:
-            if line.startswith("#") or not line.strip():
-                continue
-            k, _, v = line.partition(" ")
-            rec[k] = v.strip()
-    if rec.get("source_hash") != kernel_source_hash() or rec.get("workload") != str(workload_id):
-        return None
-    try:
-        return float(rec["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    """DRAM bytes per launch from a committed ncu record (profiles/*traffic.txt)
+    of this workload, if it was taken on the current device sources of its
+    kernel (the record's `sources` line), else None."""
+    import glob
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*traffic.txt"))):
+        rec = {}
+        with open(path) as f:
+            for line in f:
+                if line.startswith("#") or not line.strip():
+                    continue
+                k, _, v = line.partition(" ")
+                rec[k] = v.strip()
+        if rec.get("workload") != str(workload_id):
+            continue
+        sources = rec.get("sources", "").split() or None
+        if rec.get("source_hash") != kernel_source_hash(sources):
+            continue
+        try:
+            return float(rec["dram_bytes_per_launch"])
+        except (KeyError, ValueError):
+            continue
+    return None
 
 
 def algorithmic_bytes(w, k_len) -> float:
@@ -384,8 +388,8 @@ def run_ours(args, world, rank, local):
     traffic = measured_traffic(args.workload)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_src} bf16_tflops (burst)",
-                "kernel": "fa_fwd_sm100_kernel" + (" + fa_combine_kernel (split pass and merge, one event pair)"
-                                                   if splits > 1 else ""),
+                "kernel": ("fa_fwd_d256_kernel" if w.d == 256 else "fa_fwd_sm100_kernel")
+                          + (" + fa_combine_kernel (split pass and merge, one event pair)" if splits > 1 else ""),
                 "kernel_ms": kernel_ms,
                 "algorithmic_bytes": alg_bytes, "hbm_gbs_algorithmic": alg_bytes / (kernel_ms * 1e-3) / 1e9,
                 "hbm_peak_gbs": float(peaks["hbm_gbs"])}

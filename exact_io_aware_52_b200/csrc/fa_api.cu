@@ -12,6 +12,7 @@
 
 #include "fa.h"
 #include "fa_combine_kernel.cuh"
+#include "fa_fwd_d256_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 
 namespace {
@@ -24,7 +25,7 @@ struct DeviceInfo {
     bool probed = false;
     bool supported = false;
     int num_sms = 0;
-    bool attr_set[2][2] = {{false, false}, {false, false}};  // [d==128][bf16 out]
+    bool attr_set[3][2] = {};  // [d = 64, 128, 256][bf16 out]
 };
 
 std::mutex g_mu;
@@ -32,6 +33,11 @@ DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_d(int d) { return d == 64 || d == 128 || d == 256; }
+
+// Query rows per work unit: two 128-row tiles for d <= 128, one for d = 256.
+int unit_rows(int d) { return d == 256 ? fa::d256::kUnitRows : fa::kUnitRows; }
 
 fa_status load_encoder() {
     if (g_encode) return FA_OK;
@@ -91,10 +97,10 @@ fa_status validate(const fa_fwd_params *p) {
     if (p->flags & ~FA_FLAG_EAGER_RESCALE) return FA_ERR_INVALID_ARGUMENT;
     if (p->H_kv < 0 || (p->H_kv > 0 && p->H % p->H_kv != 0)) return FA_ERR_INVALID_ARGUMENT;
     if (p->N_k < 0 || p->num_splits < 0 || p->num_splits > kMaxSplits) return FA_ERR_INVALID_ARGUMENT;
-    if (p->d != 64 && p->d != 128) return FA_ERR_UNSUPPORTED;
+    if (!supported_d(p->d)) return FA_ERR_UNSUPPORTED;
     const long long rows = (long long)p->B * p->H * p->N;
     if (rows == 0) return FA_OK;
-    if ((long long)p->B * p->H > 0x7fffffffLL || (long long)p->B * p->H * ((p->N + 255) / 256) > 0x7fffffffLL)
+    if ((long long)p->B * p->H > 0x7fffffffLL || (long long)p->B * p->H * ((p->N + 127) / 128) > 0x7fffffffLL)
         return FA_ERR_INVALID_ARGUMENT;
     if (!p->q || !p->k || !p->v || !p->o || !p->lse) return FA_ERR_INVALID_ARGUMENT;
     if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v) || !aligned16(p->o)) return FA_ERR_MISALIGNED;
@@ -138,19 +144,36 @@ fa_status launch_combine(const float *o_part, const float *lse_part, void *o, fl
 
 template <int D, bool BF16>
 fa_status launch(const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t stream) {
-    auto kern = fa::fa_fwd_sm100_kernel<D, BF16>;
-    const int smem = fa::Cfg<D>::kSmemBytes;
+    constexpr bool kD256 = D == 256;
+    auto kern = kD256 ? fa::fa_fwd_d256_kernel<BF16> : fa::fa_fwd_sm100_kernel<(kD256 ? 128 : D), BF16>;
+    const int smem = kD256 ? fa::d256::kSmemBytes : fa::Cfg<(kD256 ? 128 : D)>::kSmemBytes;
+    const int threads = kD256 ? fa::d256::kThreads : fa::kThreads;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        bool &set = di.attr_set[D == 128][BF16];
+        bool &set = di.attr_set[D == 64 ? 0 : (D == 128 ? 1 : 2)][BF16];
         if (!set) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
                 return FA_ERR_CUDA;
             set = true;
         }
     }
-    kern<<<grid, fa::kThreads, smem, stream>>>(kp);
+    kern<<<grid, threads, smem, stream>>>(kp);
     return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <bool BF16>
+fa_status launch_d(int d, const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t stream) {
+    if (d == 64) return launch<64, BF16>(kp, di, grid, stream);
+    if (d == 128) return launch<128, BF16>(kp, di, grid, stream);
+    return launch<256, BF16>(kp, di, grid, stream);
+}
+
+template <bool BF16>
+fa_status launch_combine_d(int d, const float *o_part, const float *lse_part, void *o, float *lse, int splits,
+                           long long rows, int num_sms, cudaStream_t stream) {
+    if (d == 64) return launch_combine<64, BF16>(o_part, lse_part, o, lse, splits, rows, num_sms, stream);
+    if (d == 128) return launch_combine<128, BF16>(o_part, lse_part, o, lse, splits, rows, num_sms, stream);
+    return launch_combine<256, BF16>(o_part, lse_part, o, lse, splits, rows, num_sms, stream);
 }
 
 }  // namespace
@@ -200,7 +223,7 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     kp.Nk = sp.n_k;
     kp.group = p->H / H_kv;
     kp.H_kv = H_kv;
-    kp.n_blocks = (p->N + fa::kUnitRows - 1) / fa::kUnitRows;
+    kp.n_blocks = (p->N + unit_rows(p->d) - 1) / unit_rows(p->d);
     kp.n_splits = sp.splits;
     kp.split_tiles = sp.split_tiles;
     kp.n_units = BH * kp.n_blocks * sp.splits;
@@ -213,20 +236,15 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = p->o_dtype == FA_O_BF16;
     if (sp.splits > 1) {  // the split pass always writes fp32 partials; the merge writes the output type
-        st = (p->d == 64) ? launch<64, false>(kp, *di, grid, s) : launch<128, false>(kp, *di, grid, s);
-        if (st != FA_OK) return st;
-        if (p->d == 64)
-            return bf16 ? launch_combine<64, true>(o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)
-                        : launch_combine<64, false>(o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s);
-        return bf16 ? launch_combine<128, true>(o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)
-                    : launch_combine<128, false>(o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s);
+        if ((st = launch_d<false>(p->d, kp, *di, grid, s)) != FA_OK) return st;
+        return bf16 ? launch_combine_d<true>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)
+                    : launch_combine_d<false>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s);
     }
-    if (p->d == 64) return bf16 ? launch<64, true>(kp, *di, grid, s) : launch<64, false>(kp, *di, grid, s);
-    return bf16 ? launch<128, true>(kp, *di, grid, s) : launch<128, false>(kp, *di, grid, s);
+    return bf16 ? launch_d<true>(p->d, kp, *di, grid, s) : launch_d<false>(p->d, kp, *di, grid, s);
 }
 
 size_t fa_fwd_workspace_bytes(const fa_fwd_params *p) {
-    if (!p || p->num_splits <= 1 || p->B <= 0 || p->H <= 0 || p->N <= 0 || (p->d != 64 && p->d != 128)) return 0;
+    if (!p || p->num_splits <= 1 || p->B <= 0 || p->H <= 0 || p->N <= 0 || !supported_d(p->d)) return 0;
     const SplitPlan sp = plan_splits(p);
     if (sp.splits <= 1) return 0;
     const size_t rows = (size_t)p->B * p->H * p->N;
@@ -239,7 +257,8 @@ int fa_fwd_suggest_splits(const fa_fwd_params *p) {
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         return 0;
-    const long long units = (long long)p->B * p->H * ((p->N + fa::kUnitRows - 1) / fa::kUnitRows);
+    const int ur = unit_rows(supported_d(p->d) ? p->d : 128);
+    const long long units = (long long)p->B * p->H * ((p->N + ur - 1) / ur);
     const long long n_k = p->N_k > 0 ? p->N_k : p->N;
     const long long tiles = (n_k + fa::BN - 1) / fa::BN;
     if (units >= 2LL * sms || tiles <= 1) return 1;

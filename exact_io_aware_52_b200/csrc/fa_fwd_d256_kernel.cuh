@@ -1,0 +1,425 @@
+// fa_fwd_d256_kernel.cuh -- the fused exact attention forward for head
+// dimension 256 on sm_100a.
+//
+// The same computation as fa_fwd_sm100_kernel (page "FlashAttention (ES)",
+// sections "Tiling y procesamiento por bloques", "Calculo de Softmax en
+// linea" and "Fusion de operaciones en un unico kernel de CUDA"; the
+// FlashAttention-2 notes of the same page list head dimensions up to 256),
+// laid out for d = 256.  One 128-row query tile's fp32 output already fills
+// half of the 512 TMEM columns, so a work unit is one 128-row query tile of
+// one (b, h) (and one key split), and the other half of TMEM holds two score
+// buffers:
+//     S_0 [0,128), S_1 [128,256), O [256,512)
+// so that the scores of key tile j+1 are computed while the softmax works on
+// tile j.  P_j (bf16) is written over the first 64 columns of its S buffer.
+//
+// Every operand is handled as 128 x 128 bf16 half tiles (32 KB; two 64-column
+// blocks in the 128-byte-swizzle layout): Q = [Q_lo | Q_hi] along d stays in
+// shared memory for the unit; K_j and V_j stream as [lo | hi] halves through
+// one ring of five half-tile slots, loaded in the order the tensor core uses
+// them.  Products (each one tcgen05.mma group of N = 128):
+//     S_b  = Q_lo K_lo^T + Q_hi K_hi^T               (b = tile index mod 2)
+//     O_lo += P V_lo,  O_hi += P V_hi
+// Issue order in a unit with n key tiles:
+//     QK_0, QK_1, PV_0, QK_2, PV_1, QK_3, ..., PV_{n-1}
+// tcgen05.mma operations of one thread execute in issue order, so QK_{j+2}
+// overwrites P_j only after PV_j has read it, and the commit that signals
+// "S_j ready" covers PV_{j-2}.  PV_{j-1} may still run while the softmax of
+// tile j does, so when the reference maximum moves the softmax first waits for
+// PV_{j-1} (one o_done barrier per parity of the product index keeps that
+// wait exact) before it rescales O.
+//
+// Warps: 0-3 softmax (thread t owns row t of the tile), 4 MMA issuer (one
+// thread), 5 TMA producer (one thread).  192 threads, up to 255 registers each.
+#pragma once
+
+#include "fa_fwd_kernel.cuh"
+
+namespace fa {
+namespace d256 {
+
+constexpr int D = 256;
+constexpr int kUnitRows = BM;                 // one query tile per work unit
+constexpr int kHalfBytes = BM * 128 * 2;      // a 128 x 128 bf16 half tile
+constexpr int kBlockBytes = BM * 128;         // one 64-column (128-byte) block of it
+constexpr int kSlots = 5;                     // operand ring depth in half tiles
+constexpr int kSoftmaxWarps = 4;
+constexpr int kMmaWarp = 4;
+constexpr int kLoadWarp = 5;
+constexpr int kThreads = 192;
+constexpr uint32_t kColO = 256;
+
+constexpr int kOffQ = 0;                              // Q_lo, Q_hi
+constexpr int kOffRing = kOffQ + 2 * kHalfBytes;      // kSlots half tiles
+constexpr int kOffBar = kOffRing + kSlots * kHalfBytes;
+constexpr int kBarQFull = 0;
+constexpr int kBarQEmpty = 1;
+constexpr int kBarFull = 2;                     // [kSlots]
+constexpr int kBarEmpty = kBarFull + kSlots;    // [kSlots]
+constexpr int kBarSFull = kBarEmpty + kSlots;   // [2] per score buffer
+constexpr int kBarPFull = kBarSFull + 2;        // [2] per score buffer (128 arrivals)
+constexpr int kBarODone = kBarPFull + 2;        // [2] per parity of the P V product index
+constexpr int kBarOFree = kBarODone + 2;        // 128 arrivals
+constexpr int kBarDrain = kBarOFree + 1;
+constexpr int kNumBars = kBarDrain + 1;
+constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr int kOffAbort = kOffTmemSlot + 4;
+constexpr int kSmemUsed = kOffAbort + 4;
+constexpr int kSmemBytes = kSmemUsed + 1024;  // + slack to align the base to 1024 bytes
+static_assert(kHalfBytes % 1024 == 0 && kBlockBytes % 1024 == 0, "1024-byte alignment of swizzled tiles");
+static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
+static_assert(2 * kSmemBytes > 233472, "one CTA per SM: TMEM is allocated whole");
+
+// Unit t -> (b, h, query tile, split) and the key tiles [lo, lo + n) that some
+// row of the tile may attend to: as decode_unit with one query tile per unit
+// (p.n_blocks = ceil(N / 128)).
+__device__ __forceinline__ UnitCoord decode_unit1(const FwdParams &p, int t) {
+    UnitCoord u;
+    u.split = t % p.n_splits;
+    const int r = t / p.n_splits;
+    u.blk = p.n_blocks - 1 - r % p.n_blocks;
+    u.bh = r / p.n_blocks;
+    u.b = u.bh / p.H;
+    u.bh_kv = u.b * p.H_kv + (u.bh - u.b * p.H) / p.group;
+    u.lo = u.split * p.split_tiles;
+    int e = p.Nk;
+    if (p.k_len) e = min(max(__ldg(p.k_len + u.b), 0), p.Nk);
+    const int first = u.blk * kUnitRows;
+    if (p.causal) e = max(0, min(e, first + BM + (p.Nk - p.N)));
+    const int tiles = (first < p.N) ? (e + BN - 1) / BN : 0;
+    u.n[0] = max(0, min(tiles, u.lo + p.split_tiles) - u.lo);
+    u.n[1] = 0;
+    u.nmax = u.n[0];
+    return u;
+}
+
+// Waits, in order, for the completion of every P V product up to index
+// `upto` (global count over the CTA's units) not yet waited for.  Product i
+// completes phase i / 2 of o_done[i % 2]; at most one phase per barrier is
+// ever outstanding (see the issue order above), so the parity is exact.
+__device__ __forceinline__ bool wait_pv_upto(uint64_t *bars, uint32_t &waited, long long upto,
+                                             volatile int *abort_flag, uint64_t to) {
+    while ((long long)waited <= upto) {
+        if (!mbar_wait(&bars[kBarODone + (waited & 1)], (waited >> 1) & 1, abort_flag, to)) return false;
+        ++waited;
+    }
+    return true;
+}
+
+// ------------------------------------------------------------------ softmax
+template <bool O_BF16>
+__device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
+                                             uint32_t tmem, int warp, int lane) {
+    const int row_in_tile = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float LN2 = 0.69314718055994530942f;
+    const float NEG_INF = __int_as_float(0xff800000);
+    const uint32_t t_o = tmem + lane_off + kColO;
+    const uint64_t to = p.timeout_ns;
+    uint32_t gs = 0;      // score tiles consumed (global): buffer gs % 2
+    uint32_t waited = 0;  // P V products whose completion was waited for
+    uint32_t tl = 0;      // units with work (o_free phase)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+        const int t = unit_index(k);
+        if (t >= p.n_units) break;
+        const UnitCoord u = decode_unit1(p, t);
+        const int row = u.blk * kUnitRows + row_in_tile;
+        const bool row_valid = row < p.N;
+        const size_t row_id = ((size_t)u.split * p.B * p.H + u.bh) * p.N + row;
+        const int n = u.n[0];
+        if (n == 0) {  // no allowed key for these rows: O = 0, lse = -inf
+            if (row_valid) fill_row<D, O_BF16>(p.o, p.lse, row_id, false, NEG_INF);
+            continue;
+        }
+        int lim = p.Nk;  // keys [0, lim) are allowed for this row
+        if (p.k_len) lim = min(max(__ldg(p.k_len + u.b), 0), p.Nk);
+        if (p.causal) lim = min(lim, row + 1 + (p.Nk - p.N));
+
+        float m_ref = 0.f;  // reference maximum, log2 units
+        float l = 0.f;      // running sum of 2^(x - m_ref), unrounded: gives lse
+        float lr = 0.f;     // running sum of the bf16-rounded terms: O's normaliser
+        for (int j = 0; j < n; ++j, ++gs) {
+            const uint32_t buf = gs & 1;
+            const uint32_t t_s = tmem + lane_off + buf * 128u;
+            ok = mbar_wait(&bars[kBarSFull + buf], (gs >> 1) & 1, abort_flag, to);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+
+            const int kv0 = (u.lo + j) * BN;
+            const bool masked = kv0 + BN > lim;
+            float s[BN];
+            uint32_t pk0[32], pk1[32];
+            float2 ls = make_float2(0.f, 0.f);
+            float lrs = 0.f;
+            tmem_ld32f(t_s + 0, s);
+            tmem_ld32f(t_s + 32, s + 32);
+            tmem_ld32f(t_s + 64, s + 64);
+            tmem_ld32f(t_s + 96, s + 96);
+            tmem_ld_wait();
+            tmem_reg_fence_f<BN>(s);
+            if (masked) {
+                mask_scores<0>(s, kv0, lim);
+                mask_scores<1>(s, kv0, lim);
+            }
+            const float m_new = fmaxf(max64(s), max64(s + 64)) * p.scale_log2;
+            float alpha = 1.f;
+            bool resc = false;
+            if (j == 0) {
+                m_ref = (m_new == NEG_INF) ? 0.f : m_new;
+                l = 0.f;
+                lr = 0.f;
+            } else if (m_new > m_ref + p.tau) {
+                alpha = ex2_approx(m_ref - m_new);
+                l *= alpha;
+                lr *= alpha;
+                m_ref = m_new;
+                resc = true;
+            }
+            // the products before this tile's predecessor are complete (the
+            // commit behind S ready covers them): consume their phases
+            const bool any_resc = __any_sync(0xffffffffu, resc);
+            ok = wait_pv_upto(bars, waited, (long long)gs - (any_resc ? 1 : 2), abort_flag, to);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (any_resc) {
+                tc_fence_after();
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t r[32];
+                    tmem_ld32(t_o + ch * 32, r);
+                    tmem_ld_wait();
+                    tmem_reg_fence(r);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+                    tmem_st32(t_o + ch * 32, r);
+                }
+            }
+            exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
+            tmem_st32(t_s + 0, pk0);
+            exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
+            tmem_st32(t_s + 32, pk1);
+            l += ls.x + ls.y;
+            lr += lrs;
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars[kBarPFull + buf]);
+        }
+        if (ok) {
+            ok = wait_pv_upto(bars, waited, (long long)gs - 1, abort_flag, to);
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (!ok) {
+            if (row_valid) fill_row<D, O_BF16>(p.o, p.lse, row_id, true, __int_as_float(0x7fc00000));
+            break;
+        }
+        tc_fence_after();
+        const bool empty = !(lr > 0.f);
+        const float inv_l = empty ? 0.f : 1.f / lr;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(t_o + ch * 32, r);
+            tmem_ld_wait();
+            tmem_reg_fence(r);
+            if (row_valid) store_row_chunk<D, O_BF16>(p.o, row_id, ch, r, inv_l);
+        }
+        if (row_valid) p.lse[row_id] = empty ? NEG_INF : (m_ref + log2f(l)) * LN2;
+        tc_fence_before();
+        mbar_arrive(&bars[kBarOFree]);
+        ++tl;
+    }
+    return ok;
+}
+
+// ------------------------------------------------------------------ MMA issuer
+__device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
+                                         uint32_t tmem, uint32_t q_addr, uint32_t ring_addr) {
+    const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
+    const uint32_t idesc_pv = idesc_bf16_f32(BM, 128, true);
+    const uint64_t q_desc = sw128_desc(q_addr, 16, 1024);
+    const uint64_t k_desc = sw128_desc(ring_addr, 16, 1024);
+    const uint64_t v_desc = sw128_desc(ring_addr, kBlockBytes, 1024);
+    const uint64_t to = p.timeout_ns;
+    uint32_t tq = 0;   // non-empty units (q_full phase)
+    uint32_t g = 0;    // ring position
+    uint32_t gs = 0;   // score tiles issued: buffer gs % 2
+    uint32_t gpv = 0;  // P V products issued: P buffer and o_done barrier gpv % 2
+    uint32_t tl = 0;   // units with work (o_free phase)
+
+    auto take = [&](uint32_t &slot) -> bool {
+        slot = g % kSlots;
+        const bool r = mbar_wait(&bars[kBarFull + slot], (g / kSlots) & 1, abort_flag, to);
+        ++g;
+        return r;
+    };
+    auto qk = [&]() -> bool {
+        uint32_t s0, s1;
+        if (!take(s0) || !take(s1)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + (gs & 1) * 128u;
+        mma_ss_k128(d, q_desc, k_desc + ((s0 * kHalfBytes) >> 4), idesc_qk, 0u);
+        mma_ss_k128(d, q_desc + (kHalfBytes >> 4), k_desc + ((s1 * kHalfBytes) >> 4), idesc_qk, 1u);
+        tc_commit(&bars[kBarSFull + (gs & 1)]);
+        tc_commit(&bars[kBarEmpty + s0]);
+        tc_commit(&bars[kBarEmpty + s1]);
+        ++gs;
+        return true;
+    };
+    auto pv = [&](bool first) -> bool {
+        const uint32_t buf = gpv & 1;
+        if (!mbar_wait(&bars[kBarPFull + buf], (gpv >> 1) & 1, abort_flag, to)) return false;
+        if (first && tl > 0 && !mbar_wait(&bars[kBarOFree], (tl - 1) & 1, abort_flag, to)) return false;
+        uint32_t s0, s1;
+        if (!take(s0) || !take(s1)) return false;
+        tc_fence_after();
+        const uint32_t a = tmem + buf * 128u;
+        mma_ts_k128(tmem + kColO, a, v_desc + ((s0 * kHalfBytes) >> 4), idesc_pv, first ? 0u : 1u);
+        mma_ts_k128(tmem + kColO + 128u, a, v_desc + ((s1 * kHalfBytes) >> 4), idesc_pv, first ? 0u : 1u);
+        tc_commit(&bars[kBarODone + buf]);
+        tc_commit(&bars[kBarEmpty + s0]);
+        tc_commit(&bars[kBarEmpty + s1]);
+        ++gpv;
+        return true;
+    };
+
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+        const int t = unit_index(k);
+        if (t >= p.n_units) break;
+        const UnitCoord u = decode_unit1(p, t);
+        const int n = u.n[0];
+        if (n == 0) continue;
+        if (!mbar_wait(&bars[kBarQFull], tq & 1, abort_flag, to)) { ok = false; break; }
+        ++tq;
+        tc_fence_after();
+        int jq = 0;  // score tiles of this unit issued
+        auto qk_next = [&]() -> bool {
+            if (!qk()) return false;
+            if (++jq == n) tc_commit(&bars[kBarQEmpty]);  // Q no longer read in this unit
+            return true;
+        };
+        if (!qk_next()) { ok = false; break; }
+        if (n > 1 && !qk_next()) { ok = false; break; }
+        for (int j = 0; j < n; ++j) {
+            if (!pv(j == 0)) { ok = false; break; }
+            if (j + 2 < n && !qk_next()) { ok = false; break; }
+        }
+        ++tl;
+    }
+    return ok;
+}
+
+// ------------------------------------------------------------------ TMA producer
+__device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
+                                          uint8_t *sQ, uint8_t *ring) {
+    prefetch_tensormap(&p.tm_q);
+    prefetch_tensormap(&p.tm_k);
+    prefetch_tensormap(&p.tm_v);
+    const uint64_t to = p.timeout_ns;
+    uint32_t tq = 0, g = 0;
+    bool ok = true;
+    // key tile `kt` of K or V as two half tiles (d columns [0,128) and [128,256))
+    auto load_tile = [&](const CUtensorMap *map, int kt, int bh_kv) -> bool {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t slot = g % kSlots, round = g / kSlots;
+            if (round > 0 && !mbar_wait(&bars[kBarEmpty + slot], (round - 1) & 1, abort_flag, to)) return false;
+            mbar_arrive_expect_tx(&bars[kBarFull + slot], kHalfBytes);
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+                tma_load_3d(ring + slot * kHalfBytes + c * kBlockBytes, map, &bars[kBarFull + slot], h * 128 + c * 64,
+                            kt * BN, bh_kv);
+            ++g;
+        }
+        return true;
+    };
+    for (int k = 0; ok; ++k) {
+        const int t = unit_index(k);
+        if (t >= p.n_units) break;
+        const UnitCoord u = decode_unit1(p, t);
+        const int n = u.n[0];
+        if (n == 0) continue;
+        if (tq > 0 && !mbar_wait(&bars[kBarQEmpty], (tq - 1) & 1, abort_flag, to)) {
+            ok = false;
+            break;
+        }
+        mbar_arrive_expect_tx(&bars[kBarQFull], 2 * kHalfBytes);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            tma_load_3d(sQ + c * kBlockBytes, &p.tm_q, &bars[kBarQFull], c * 64, u.blk * kUnitRows, u.bh);
+        ++tq;
+        // the order the MMA issuer takes them: K_0, K_1, V_0, K_2, V_1, ..., V_{n-1}
+        if (!load_tile(&p.tm_k, u.lo, u.bh_kv)) { ok = false; break; }
+        if (n > 1 && !load_tile(&p.tm_k, u.lo + 1, u.bh_kv)) { ok = false; break; }
+        for (int j = 0; j < n && ok; ++j) {
+            if (!load_tile(&p.tm_v, u.lo + j, u.bh_kv)) ok = false;
+            else if (j + 2 < n && !load_tile(&p.tm_k, u.lo + j + 2, u.bh_kv)) ok = false;
+        }
+    }
+    if (!ok) record_timeout(p);
+    // drain: every copy this thread issued has landed before the CTA may exit
+    if (tq > 0) mbar_wait_drain(&bars[kBarQFull], (tq - 1) & 1, to);
+    const uint32_t nr = g < (uint32_t)kSlots ? g : (uint32_t)kSlots;
+    for (uint32_t i = 0; i < nr; ++i) {
+        const uint32_t gi = g - 1 - i;
+        mbar_wait_drain(&bars[kBarFull + gi % kSlots], (gi / kSlots) & 1, to);
+    }
+}
+
+}  // namespace d256
+
+template <bool O_BF16>
+__global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_d256_kernel(const __grid_constant__ FwdParams p) {
+    using namespace d256;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *sQ = smem + kOffQ;
+    uint8_t *ring = smem + kOffRing;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmemSlot);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNumBars; ++i) {
+            const bool per_row = (i >= kBarPFull && i < kBarPFull + 2) || i == kBarOFree;
+            mbar_init(&bars[i], per_row ? 128u : 1u);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == d256::kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < d256::kSoftmaxWarps) {
+        if (!d256::softmax_role<O_BF16>(p, bars, abort_flag, tmem, warp, lane)) record_timeout(p);
+    } else if (warp == d256::kMmaWarp) {
+        if (lane == 0) {
+            if (!d256::mma_role(p, bars, abort_flag, tmem, smem_u32(sQ), smem_u32(ring))) record_timeout(p);
+            tc_commit(&bars[kBarDrain]);
+            mbar_wait_drain(&bars[kBarDrain], 0, p.timeout_ns);
+        }
+    } else if (warp == d256::kLoadWarp) {
+        if (lane == 0) d256::load_role(p, bars, abort_flag, sQ, ring);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == d256::kMmaWarp) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace fa

@@ -77,6 +77,9 @@ WORKLOADS = {
     # cached keys: 256 new queries per head against 128K keys, key range split across SMs
     7: Workload("cached-keys causal grouped-KV B1 H32 Hkv8 Nq256 Nk131072 d128 split-KV", 1, 32, 256, 128, True,
                 sample_rows_per_head=16, seed=52007, H_kv=8, Nk=131072, splits=-1),
+    # head dimension 256: the FLOPs of workload 4 with half the heads
+    8: Workload("long-context causal B1 H16 N16384 d256", 1, 16, 16384, 256, True,
+                sample_rows_per_head=256, seed=52008),
 }
 
 

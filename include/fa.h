@@ -59,7 +59,7 @@ typedef enum {
     FA_OK = 0,
     FA_ERR_INVALID_ARGUMENT = 1, /* NULL pointer, negative size, bad scale, bad dtype */
     FA_ERR_MISALIGNED = 2,       /* a pointer not 16-byte aligned (TMA requirement)   */
-    FA_ERR_UNSUPPORTED = 3,      /* d not in {64, 128}, or the device is not sm_100    */
+    FA_ERR_UNSUPPORTED = 3,      /* d not in {64, 128, 256}, or the device is not sm_100 */
     FA_ERR_CUDA = 4,             /* a CUDA runtime/driver call or the launch failed   */
     FA_ERR_DEVICE_TIMEOUT = 5,   /* (device status word) a pipeline wait timed out     */
     FA_ERR_WORKSPACE_LIMIT = 6   /* fa_fwd_static_workspace: the splits need more than
@@ -83,7 +83,7 @@ enum {
  *   o       : device fp32 [B, H, N, d], 16-byte aligned
  *   lse     : device fp32 [B, H, N]
  *   B, H, N : >= 0 (B*H*N == 0 is a no-op returning FA_OK)
- *   d       : 64 or 128
+ *   d       : 64, 128 or 256
  *   causal  : 0 or 1
  *   scale   : finite, > 0 (the definition's 1/sqrt(d_k))
  *   stream  : cudaStream_t

@@ -85,7 +85,8 @@ def _ex(**kw):
     (dict(N_k=1024, num_splits=4, workspace=0x80000, workspace_bytes=64), fb.FA_ERR_INVALID_ARGUMENT),
     (dict(N_k=1024, num_splits=4, workspace=0x80008, workspace_bytes=1 << 30), fb.FA_ERR_MISALIGNED),
     (dict(d=32), fb.FA_ERR_UNSUPPORTED),
-    (dict(d=256), fb.FA_ERR_UNSUPPORTED),
+    (dict(d=512), fb.FA_ERR_UNSUPPORTED),
+    (dict(d=192), fb.FA_ERR_UNSUPPORTED),
     (dict(d=96), fb.FA_ERR_UNSUPPORTED),
     (dict(q=0x10008), fb.FA_ERR_MISALIGNED),
     (dict(k=0x20004), fb.FA_ERR_MISALIGNED),

@@ -11,6 +11,10 @@ Two pieces, both written from the page "FlashAttention (ES)":
   section "Fusion de operaciones en un unico kernel de CUDA"), computed in C
   with OpenMP over rows in ``attn_oracle.c``: full score row, mask,
   max-subtracted softmax, weighted sum of V rows.
+* ``attention_bwd_f64`` -- the gradients dQ, dK, dV of that definition for a
+  given dO (the chain rule through the row softmax; the pages give no
+  backward algorithm), in C with OpenMP over key/value heads in
+  ``attn_bwd_oracle.c``.
 * ``online.attention_online`` -- the tiled online-softmax recurrence of
   section "Calculo de Softmax en linea" in pure Python, used only on tiny
   inputs to pin the recurrence against the two-pass definition.
@@ -30,8 +34,11 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "attn_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+_BWD_SRC = os.path.join(_HERE, "attn_bwd_oracle.c")
+_BWD_LIB = os.path.join(_HERE, "liboracle_bwd.so")
 _lock = threading.Lock()
 _lib = None
+_bwd_lib = None
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
@@ -66,6 +73,29 @@ def _load():
         if _lib is None:
             _lib = load_library(build())
     return _lib
+
+
+def build_bwd(force: bool = False, src: str = _BWD_SRC, out: str = _BWD_LIB) -> str:
+    """Compile the backward oracle (``attn_bwd_oracle.c`` by default)."""
+    return build(force=force, src=src, out=out)
+
+
+def load_bwd_library(path: str):
+    """ctypes handle on a built backward-oracle library with its signature declared."""
+    lib = ctypes.CDLL(path)
+    f = lib.attn_bwd_oracle_f64
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 + [ctypes.c_float] + [ctypes.c_void_p] * 3 + \
+        [ctypes.c_int]
+    return lib
+
+
+def _load_bwd():
+    global _bwd_lib
+    with _lock:
+        if _bwd_lib is None:
+            _bwd_lib = load_bwd_library(build_bwd())
+    return _bwd_lib
 
 
 def _as_bf16_bits(x) -> np.ndarray:
@@ -125,3 +155,38 @@ def attention_f64(q, k, v, causal: bool, scale: float, k_len=None, rows=None,
     if rc != 0:
         raise RuntimeError(f"attn_oracle_f64 failed with code {rc}")
     return o, lse
+
+
+def attention_bwd_f64(q, k, v, dout, causal: bool, scale: float, k_len=None, nthreads: int | None = None,
+                      lib=None):
+    """Gradients of exact attention in fp64 from bf16 inputs.
+
+    q, dout: [B, H, N, d]; k, v: [B, H_kv, Nk, d] (bf16 torch CPU tensors or
+    uint16 bit arrays), with the masks and head grouping of ``attention_f64``;
+    dout is the gradient of the loss with respect to O.
+    Returns (dq [B, H, N, d], dk [B, H_kv, Nk, d], dv [B, H_kv, Nk, d]) float64.
+    """
+    qb, kb, vb, db = _as_bf16_bits(q), _as_bf16_bits(k), _as_bf16_bits(v), _as_bf16_bits(dout)
+    if qb.ndim != 4 or kb.shape != vb.shape or db.shape != qb.shape:
+        raise ValueError("q, dout must be [B, H, N, d] and k, v [B, H_kv, Nk, d]")
+    B, H, N, d = qb.shape
+    H_kv, Nk = kb.shape[1], kb.shape[2]
+    if (kb.shape[0], kb.shape[3]) != (B, d) or H_kv == 0 or H % H_kv:
+        raise ValueError("k, v must be [B, H_kv, Nk, d] with H_kv dividing H")
+    kl = None
+    if k_len is not None:
+        kl = np.ascontiguousarray(np.asarray(k_len, dtype=np.int32).reshape(-1))
+        if kl.shape[0] != B:
+            raise ValueError("k_len must have B entries")
+    dq = np.zeros((B, H, N, d), dtype=np.float64)
+    dk = np.zeros((B, H_kv, Nk, d), dtype=np.float64)
+    dv = np.zeros((B, H_kv, Nk, d), dtype=np.float64)
+    nt = nthreads if nthreads is not None else (os.cpu_count() or 1)
+    lib = _load_bwd() if lib is None else lib
+    rc = lib.attn_bwd_oracle_f64(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, db.ctypes.data,
+        None if kl is None else kl.ctypes.data, B, H, H_kv, N, Nk, d, int(bool(causal)),
+        ctypes.c_float(scale), dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, int(nt))
+    if rc != 0:
+        raise RuntimeError(f"attn_bwd_oracle_f64 failed with code {rc}")
+    return dq, dk, dv

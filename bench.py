@@ -103,8 +103,9 @@ def algorithmic_bytes(w, k_len) -> float:
     """Compulsory HBM bytes of one launch: Q, K, V read once (valid keys only
     under key padding), O (fp32) and lse written once."""
     n_elem = w.B * w.H * w.N * w.d
+    eb = 1.0 if w.dtype == "e4m3" else 2.0
     kv_rows = w.kv_heads * (sum(min(max(int(x), 0), w.keys) for x in k_len) if k_len is not None else w.B * w.keys)
-    return 2.0 * n_elem + 2 * 2.0 * kv_rows * w.d + 4.0 * n_elem + 4.0 * w.B * w.H * w.N
+    return eb * n_elem + 2 * eb * kv_rows * w.d + 4.0 * n_elem + 4.0 * w.B * w.H * w.N
 
 
 class ClockSampler:
@@ -227,12 +228,18 @@ def oracle_rows_flops(w, rows, k_len) -> float:
     return 4.0 * w.d * tot
 
 
+def exact_bf16(t):
+    """E4M3 inputs widened exactly to bf16 (the oracle reads bf16); others as they are."""
+    return t.to(torch.bfloat16) if t.dtype == torch.float8_e4m3fn else t
+
+
 def cpu_oracle_rate(w, q, k, v, k_len, budget_s: float, seed: int = 0):
     """Time the fp64 oracle on rows of the workload for about budget_s seconds;
     returns (TFLOP/s in the metric's unit, threads, description, seconds)."""
     import numpy as np
 
     import oracle
+    q, k, v = exact_bf16(q), exact_bf16(k), exact_bf16(v)
     threads = os.cpu_count() or 1
     rng = np.random.default_rng(seed)
     n_rows = w.B * w.H * w.N
@@ -266,9 +273,11 @@ def run_reference(args, world, rank):
     rows_per_step = max(threads, 8)
     n_rows = w.B * w.H * w.N
 
+    qo, ko, vo = exact_bf16(q), exact_bf16(k), exact_bf16(v)
+
     def step():
         rows = np.sort(rng.choice(n_rows, size=rows_per_step, replace=False)).astype(np.int64)
-        oracle.attention_f64(q, k, v, w.causal, w.scale, k_len=kl, rows=rows, nthreads=threads)
+        oracle.attention_f64(qo, ko, vo, w.causal, w.scale, k_len=kl, rows=rows, nthreads=threads)
         return oracle_rows_flops(w, rows, kl)
 
     for _ in range(args.warmup):
@@ -283,7 +292,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, world, (q.numel() + k.numel() + v.numel()) * 2),
+        "config": workload_config(w, world, (q.numel() + k.numel() + v.numel()) * q.element_size()),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"each step: the fp64 oracle on {rows_per_step} uniformly sampled query "
                                    f"rows of the workload (all keys of each row); {args.steps} steps"},
@@ -373,7 +382,7 @@ def run_ours(args, world, rank, local):
         e1.record(stream)
         e1.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-        h2d = (qh.numel() + kh.numel() + vh.numel()) * 2 + (0 if klh is None else klh.numel() * 4)
+        h2d = (qh.numel() + kh.numel() + vh.numel()) * qh.element_size() + (0 if klh is None else klh.numel() * 4)
         d2h = oh.numel() * 4 + lh.numel() * 4
         e2e = {"value": flops * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
@@ -383,11 +392,13 @@ def run_ours(args, world, rank, local):
         return
     peaks, peak_src = load_peaks()
     achieved = flops / (kernel_ms * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops"])
+    # E4M3 products: the measured bf16 peak times the nominal dense FP8 / BF16 ratio (4.5 / 2.25)
+    fp8 = w.dtype == "e4m3"
+    peak = float(peaks["bf16_tflops"]) * (2.0 if fp8 else 1.0)
     alg_bytes = algorithmic_bytes(w, k_len)
     traffic = measured_traffic(args.workload)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_src} bf16_tflops (burst)" + (" x 2 (nominal FP8/BF16 dense ratio)" if fp8 else ""),
                 "kernel": ("fa_fwd_d256_kernel" if w.d == 256 else "fa_fwd_sm100_kernel")
                           + (" + fa_combine_kernel (split pass and merge, one event pair)" if splits > 1 else ""),
                 "kernel_ms": kernel_ms,
@@ -400,8 +411,8 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w, world, (q.numel() + k.numel() + v.numel()) * 2),
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
+        "config": workload_config(w, world, (q.numel() + k.numel() + v.numel()) * q.element_size()),
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": roofline,
         "cpu_baseline": cpu,

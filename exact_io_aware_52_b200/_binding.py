@@ -25,6 +25,8 @@ FA_ERR_WORKSPACE_LIMIT = 6
 FA_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024   # include/fa.h
 FA_O_F32 = 0
 FA_O_BF16 = 1
+FA_IN_BF16 = 0
+FA_IN_E4M3 = 1
 FA_FLAG_EAGER_RESCALE = 1
 
 _lock = threading.Lock()
@@ -42,7 +44,8 @@ class FaParams(ctypes.Structure):
         ("causal", ctypes.c_int), ("scale", ctypes.c_float), ("o_dtype", ctypes.c_int),
         ("flags", ctypes.c_int), ("timeout_ms", ctypes.c_uint32), ("H_kv", ctypes.c_int),
         ("N_k", ctypes.c_int), ("num_splits", ctypes.c_int), ("workspace", ctypes.c_void_p),
-        ("workspace_bytes", ctypes.c_size_t),
+        ("workspace_bytes", ctypes.c_size_t), ("in_dtype", ctypes.c_int), ("descale_q", ctypes.c_float),
+        ("descale_k", ctypes.c_float), ("descale_v", ctypes.c_float),
     ]
 
 
@@ -108,6 +111,10 @@ def load_selftest():
             lib.fa_selftest_mma_ss.argtypes = [vp, vp, vp, i, vp, vp]
             lib.fa_selftest_mma_ts.restype = i
             lib.fa_selftest_mma_ts.argtypes = [vp, vp, vp, i, vp, vp]
+            lib.fa_selftest_mma_e4m3_ss.restype = i
+            lib.fa_selftest_mma_e4m3_ss.argtypes = [vp, vp, vp, vp, vp]
+            lib.fa_selftest_mma_e4m3_ts.restype = i
+            lib.fa_selftest_mma_e4m3_ts.argtypes = [vp, vp, vp, vp, vp]
             lib.fa_selftest_exp2_poly.restype = i
             lib.fa_selftest_exp2_poly.argtypes = [vp, vp, i, vp]
             lib.fa_selftest_wait_timeout.restype = i
@@ -151,11 +158,13 @@ def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
 
 
 def make_params(q, k, v, o, lse, causal, scale, k_len=None, dev_status=None, flags=0, timeout_ms=0,
-                shape=None, num_splits=0, workspace=None) -> FaParams:
+                shape=None, num_splits=0, workspace=None, descale=(0.0, 0.0, 0.0)) -> FaParams:
     """Fill a fa_fwd_params from tensors (any of them may be None for argument tests).
 
     k, v may be [B, H_kv, N_k, d] with H_kv dividing H and any N_k; workspace is a
-    CUDA tensor of at least workspace_bytes(...) bytes when num_splits > 1."""
+    CUDA tensor of at least workspace_bytes(...) bytes when num_splits > 1.
+    q, k, v of dtype torch.float8_e4m3fn select E4M3 inputs, whose values are
+    scaled by descale = (descale_q, descale_k, descale_v) (0 means 1)."""
     import torch
     if shape is None:
         shape = tuple(q.shape)
@@ -172,7 +181,9 @@ def make_params(q, k, v, o, lse, causal, scale, k_len=None, dev_status=None, fla
                     dev_status=_ptr(dev_status), B=B, H=H, N=N, d=d, causal=int(bool(causal)),
                     scale=float(scale), o_dtype=o_dtype, flags=int(flags), timeout_ms=int(timeout_ms),
                     H_kv=H_kv, N_k=N_k, num_splits=int(num_splits), workspace=_ptr(workspace),
-                    workspace_bytes=ws_bytes)
+                    workspace_bytes=ws_bytes,
+                    in_dtype=FA_IN_E4M3 if getattr(q, "dtype", None) == torch.float8_e4m3fn else FA_IN_BF16,
+                    descale_q=float(descale[0]), descale_k=float(descale[1]), descale_v=float(descale[2]))
 
 
 def workspace_bytes(q, k, num_splits: int) -> int:
@@ -188,31 +199,33 @@ def suggest_splits(q, k) -> int:
 
 
 def fa_fwd_ex(q, k, v, o, lse, causal: bool, scale: float, k_len=None, dev_status=None, flags: int = 0,
-              timeout_ms: int = 0, stream=None, num_splits: int = 0, workspace=None):
+              timeout_ms: int = 0, stream=None, num_splits: int = 0, workspace=None, descale=(0.0, 0.0, 0.0)):
     """fa_fwd_ex: as fa_fwd, plus k_len (int32 [B] CUDA tensor), o may be bf16,
     an optional int32 status word, FA_FLAG_* flags and the wait time limit.
     k and v may be [B, H_kv, N_k, d] (grouped heads, more keys than queries);
     num_splits > 1 splits each row's keys, with `workspace` as scratch."""
     p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms,
-                    num_splits=num_splits, workspace=workspace)
+                    num_splits=num_splits, workspace=workspace, descale=descale)
     _check(load().fa_fwd_ex(ctypes.byref(p), _stream(stream)), "fa_fwd_ex")
 
 
 def fa_fwd_static_workspace(q, k, v, o, lse, causal: bool, scale: float, k_len=None, dev_status=None,
-                            flags: int = 0, timeout_ms: int = 0, stream=None, num_splits: int = 0):
+                            flags: int = 0, timeout_ms: int = 0, stream=None, num_splits: int = 0,
+                            descale=(0.0, 0.0, 0.0)):
     """fa_fwd_static_workspace: fa_fwd_ex with the split scratch in the library's
     fixed device array (FA_STATIC_WORKSPACE_BYTES per device, shared by all calls
     on the device: do not overlap calls).  Allocates nothing."""
-    p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms, num_splits=num_splits)
+    p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms, num_splits=num_splits,
+                    descale=descale)
     _check(load().fa_fwd_static_workspace(ctypes.byref(p), _stream(stream)), "fa_fwd_static_workspace")
 
 
 def fa_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal: bool, scale: float,
                 k_len_h=None, k_len_d=None, dev_status=None, flags: int = 0, stream=None, num_splits: int = 0,
-                workspace=None):
+                workspace=None, descale=(0.0, 0.0, 0.0)):
     """fa_fwd_host: host (pinned) tensors in and out, device tensors as staging."""
     dev = make_params(q_d, k_d, v_d, o_d, lse_d, causal, scale, k_len_d, dev_status, flags,
-                      num_splits=num_splits, workspace=workspace)
+                      num_splits=num_splits, workspace=workspace, descale=descale)
     hp = FaHostParams(q=_ptr(q_h), k=_ptr(k_h), v=_ptr(v_h), k_len=_ptr(k_len_h), o=_ptr(o_h), lse=_ptr(lse_h),
                       dev=dev)
     _check(load().fa_fwd_host(ctypes.byref(hp), _stream(stream)), "fa_fwd_host")
@@ -223,7 +236,7 @@ def read_device_status(dev_status, stream=None) -> int:
 
 
 def attention(q, k, v, causal: bool, scale: float, k_len=None, out_dtype=None, flags: int = 0, stream=None,
-              num_splits: int = 0):
+              num_splits: int = 0, descale=(0.0, 0.0, 0.0)):
     """Allocate O, lse (and any split workspace) with torch on q's device and run fa_fwd_ex.
 
     num_splits: 0 = none, -1 = the library's suggestion, S > 1 = S key splits.
@@ -239,5 +252,5 @@ def attention(q, k, v, causal: bool, scale: float, k_len=None, out_dtype=None, f
     if num_splits > 1:
         ws = torch.empty(max(workspace_bytes(q, k, num_splits), 16), dtype=torch.uint8, device=q.device)
     fa_fwd_ex(q, k, v, o, lse, causal, scale, k_len=k_len, flags=flags, stream=stream, num_splits=num_splits,
-              workspace=ws)
+              workspace=ws, descale=descale)
     return o, lse

@@ -17,7 +17,7 @@
 
 namespace {
 
-constexpr int kVersion = 200;  // 0.2.0
+constexpr int kVersion = 300;  // 0.3.0
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplits = 1024;
 
@@ -25,7 +25,7 @@ struct DeviceInfo {
     bool probed = false;
     bool supported = false;
     int num_sms = 0;
-    bool attr_set[3][2] = {};  // [d = 64, 128, 256][bf16 out]
+    bool attr_set[4][2] = {};  // [d = 64, 128, 256, 128 with E4M3 inputs][bf16 out]
 };
 
 std::mutex g_mu;
@@ -35,6 +35,11 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool supported_d(int d) { return d == 64 || d == 128 || d == 256; }
+
+bool e4m3_in(const fa_fwd_params *p) { return p->in_dtype == FA_IN_E4M3; }
+
+bool valid_descale(float x) { return std::isfinite(x) && x >= 0.f; }
+float descale(float x) { return x > 0.f ? x : 1.f; }
 
 // Query rows per work unit: two 128-row tiles for d <= 128, one for d = 256.
 int unit_rows(int d) { return d == 256 ? fa::d256::kUnitRows : fa::kUnitRows; }
@@ -72,16 +77,18 @@ fa_status probe_device(int *dev_out, DeviceInfo **info_out) {
     return FA_OK;
 }
 
-// 3-D map over a contiguous [B*H][N][D] bf16 tensor: dims innermost first
-// {D, N, B*H}; box {64, 128, 1} (one 128-byte column block of a 128-row
+// 3-D map over a contiguous [B*H][N][D] tensor of bf16 (elem_bytes 2) or
+// E4M3 (elem_bytes 1, mapped as bytes): dims innermost first {D, N, B*H};
+// box {128 / elem_bytes, 128, 1} (one 128-byte column block of a 128-row
 // tile); 128-byte swizzle, the layout the tcgen05 descriptors describe.
 // Out-of-range rows read as zero.
-fa_status encode_map(CUtensorMap *map, const void *base, int BH, int N, int D) {
+fa_status encode_map(CUtensorMap *map, const void *base, int BH, int N, int D, int elem_bytes = 2) {
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)fa::BM, 1};
+    cuuint64_t strides[2] = {(cuuint64_t)D * elem_bytes, (cuuint64_t)N * D * elem_bytes};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / elem_bytes), (cuuint32_t)fa::BM, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+    const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = g_encode(map, dt, 3, const_cast<void *>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
@@ -97,7 +104,11 @@ fa_status validate(const fa_fwd_params *p) {
     if (p->flags & ~FA_FLAG_EAGER_RESCALE) return FA_ERR_INVALID_ARGUMENT;
     if (p->H_kv < 0 || (p->H_kv > 0 && p->H % p->H_kv != 0)) return FA_ERR_INVALID_ARGUMENT;
     if (p->N_k < 0 || p->num_splits < 0 || p->num_splits > kMaxSplits) return FA_ERR_INVALID_ARGUMENT;
+    if (p->in_dtype != FA_IN_BF16 && p->in_dtype != FA_IN_E4M3) return FA_ERR_INVALID_ARGUMENT;
+    if (!valid_descale(p->descale_q) || !valid_descale(p->descale_k) || !valid_descale(p->descale_v))
+        return FA_ERR_INVALID_ARGUMENT;
     if (!supported_d(p->d)) return FA_ERR_UNSUPPORTED;
+    if (e4m3_in(p) && p->d != 128) return FA_ERR_UNSUPPORTED;
     const long long rows = (long long)p->B * p->H * p->N;
     if (rows == 0) return FA_OK;
     if ((long long)p->B * p->H > 0x7fffffffLL || (long long)p->B * p->H * ((p->N + 127) / 128) > 0x7fffffffLL)
@@ -142,15 +153,16 @@ fa_status launch_combine(const float *o_part, const float *lse_part, void *o, fl
     return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool F8 = false>
 fa_status launch(const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t stream) {
     constexpr bool kD256 = D == 256;
-    auto kern = kD256 ? fa::fa_fwd_d256_kernel<BF16> : fa::fa_fwd_sm100_kernel<(kD256 ? 128 : D), BF16>;
-    const int smem = kD256 ? fa::d256::kSmemBytes : fa::Cfg<(kD256 ? 128 : D)>::kSmemBytes;
+    constexpr int kD = kD256 ? 128 : D;
+    auto kern = kD256 ? fa::fa_fwd_d256_kernel<BF16> : fa::fa_fwd_sm100_kernel<kD, BF16, F8>;
+    const int smem = kD256 ? fa::d256::kSmemBytes : fa::Cfg<kD, F8>::kSmemBytes;
     const int threads = kD256 ? fa::d256::kThreads : fa::kThreads;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        bool &set = di.attr_set[D == 64 ? 0 : (D == 128 ? 1 : 2)][BF16];
+        bool &set = di.attr_set[F8 ? 3 : (D == 64 ? 0 : (D == 128 ? 1 : 2))][BF16];
         if (!set) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
                 return FA_ERR_CUDA;
@@ -162,7 +174,8 @@ fa_status launch(const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t
 }
 
 template <bool BF16>
-fa_status launch_d(int d, const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t stream) {
+fa_status launch_d(int d, bool e4m3, const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t stream) {
+    if (e4m3) return launch<128, BF16, true>(kp, di, grid, stream);
     if (d == 64) return launch<64, BF16>(kp, di, grid, stream);
     if (d == 128) return launch<128, BF16>(kp, di, grid, stream);
     return launch<256, BF16>(kp, di, grid, stream);
@@ -199,11 +212,12 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     const int BH = p->B * p->H;
     const int H_kv = p->H_kv > 0 ? p->H_kv : p->H;
     const SplitPlan sp = plan_splits(p);
-    if ((st = encode_map(&kp.tm_q, p->q, BH, p->N, p->d)) != FA_OK) return st;
+    const int eb = e4m3_in(p) ? 1 : 2;
+    if ((st = encode_map(&kp.tm_q, p->q, BH, p->N, p->d, eb)) != FA_OK) return st;
     // a map over zero keys is not encodable; with N_k = 0 no key tile is loaded
     const int n_k_map = sp.n_k > 0 ? sp.n_k : 1;
-    if ((st = encode_map(&kp.tm_k, p->k, p->B * H_kv, n_k_map, p->d)) != FA_OK) return st;
-    if ((st = encode_map(&kp.tm_v, p->v, p->B * H_kv, n_k_map, p->d)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_k, p->k, p->B * H_kv, n_k_map, p->d, eb)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_v, p->v, p->B * H_kv, n_k_map, p->d, eb)) != FA_OK) return st;
     const long long rows = (long long)BH * p->N;
     float *o_part = nullptr, *lse_part = nullptr;
     if (sp.splits > 1) {  // partials: fp32 [S][rows][d], then fp32 [S][rows]
@@ -228,19 +242,30 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     kp.split_tiles = sp.split_tiles;
     kp.n_units = BH * kp.n_blocks * sp.splits;
     kp.causal = p->causal;
-    kp.scale_log2 = (float)((double)p->scale * 1.4426950408889634074);
-    kp.tau = (p->flags & FA_FLAG_EAGER_RESCALE) ? 0.f : 8.f;
+    if (e4m3_in(p)) {
+        // value scales: Q K^T by descale_q * descale_k (folded into the softmax
+        // scale), O by descale_v; eager rescaling keeps P in E4M3's normal range
+        kp.scale_log2 = (float)((double)p->scale * descale(p->descale_q) * descale(p->descale_k) *
+                                1.4426950408889634074);
+        kp.tau = 0.f;
+        kp.out_scale = descale(p->descale_v);
+    } else {
+        kp.scale_log2 = (float)((double)p->scale * 1.4426950408889634074);
+        kp.tau = (p->flags & FA_FLAG_EAGER_RESCALE) ? 0.f : 8.f;
+        kp.out_scale = 1.f;
+    }
     kp.timeout_ns = (uint64_t)(p->timeout_ms ? p->timeout_ms : 2000u) * 1000000ull;
 
     const int grid = kp.n_units < di->num_sms ? kp.n_units : di->num_sms;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = p->o_dtype == FA_O_BF16;
     if (sp.splits > 1) {  // the split pass always writes fp32 partials; the merge writes the output type
-        if ((st = launch_d<false>(p->d, kp, *di, grid, s)) != FA_OK) return st;
+        if ((st = launch_d<false>(p->d, e4m3_in(p), kp, *di, grid, s)) != FA_OK) return st;
         return bf16 ? launch_combine_d<true>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)
                     : launch_combine_d<false>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s);
     }
-    return bf16 ? launch_d<true>(p->d, kp, *di, grid, s) : launch_d<false>(p->d, kp, *di, grid, s);
+    return bf16 ? launch_d<true>(p->d, e4m3_in(p), kp, *di, grid, s)
+                : launch_d<false>(p->d, e4m3_in(p), kp, *di, grid, s);
 }
 
 size_t fa_fwd_workspace_bytes(const fa_fwd_params *p) {
@@ -314,9 +339,10 @@ fa_status fa_fwd_host(const fa_fwd_host_params *hp, void *stream) {
     if (!hp->q || !hp->k || !hp->v || !hp->o || !hp->lse) return FA_ERR_INVALID_ARGUMENT;
     if ((hp->k_len == nullptr) != (p->k_len == nullptr)) return FA_ERR_INVALID_ARGUMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const size_t q_bytes = rows * p->d * 2;
+    const size_t eb = e4m3_in(p) ? 1 : 2;
+    const size_t q_bytes = rows * p->d * eb;
     const size_t kv_bytes =
-        (size_t)p->B * (p->H_kv > 0 ? p->H_kv : p->H) * (p->N_k > 0 ? p->N_k : p->N) * p->d * 2;
+        (size_t)p->B * (p->H_kv > 0 ? p->H_kv : p->H) * (p->N_k > 0 ? p->N_k : p->N) * p->d * eb;
     const size_t o_bytes = rows * p->d * (p->o_dtype == FA_O_BF16 ? 2 : 4);
     if (cudaMemcpyAsync(const_cast<void *>(p->q), hp->q, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(const_cast<void *>(p->k), hp->k, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||

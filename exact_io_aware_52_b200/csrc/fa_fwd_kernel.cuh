@@ -77,6 +77,15 @@ constexpr int kPolyPairs = 0;
 // P to bf16: round to nearest even (cvt) when false; truncation (keep the
 // high half of each fp32 word, one byte permute per pair) when true.
 constexpr bool kPackTruncate = false;
+// P V in two halves of 64 keys: the softmax releases P for keys [0, 64) as
+// soon as it is in TMEM, so the tensor core multiplies that half while the
+// softmax computes the other, and only P V for keys [64, 128) plus the next
+// Q K^T remain between "P ready" and the next "S ready".  Measured on B200
+// (300 launches each): d = 64 (B8 H12 N1024 causal) 48.5 -> 47.1 us; d = 128
+// (B1 H32 N16384 causal) 2.249 -> 2.306 ms, where the extra store wait in the
+// middle of the softmax costs more than the overlap gains.  On for d = 64 only.
+template <int D>
+constexpr bool kSplitPV = (D == 64);
 
 __device__ __forceinline__ uint32_t col_s(uint32_t x) { return x * 128u; }                  // S_X, P_X
 __device__ __forceinline__ uint32_t col_o(uint32_t x, uint32_t d) { return 256u + x * d; }  // O_X
@@ -99,16 +108,22 @@ struct FwdParams {
     int causal;
     float scale_log2;              // scale * log2(e)
     float tau;                     // rescale threshold in log2 units (<= 0: rescale on any growth)
+    float out_scale;               // factor on O (the value scale of E4M3 inputs; 1 for bf16)
     uint64_t timeout_ns;
 };
 
-template <int D>
+// F8: Q, K and V in E4M3 (one byte per element, d = 128 only), products on
+// tcgen05 kind::f8f6f4; otherwise bf16 and kind::f16.
+template <int D, bool F8 = false>
 struct Cfg {
-    static constexpr int kChunks = D / 64;          // 64-element (128-byte) column blocks per row
-    static constexpr int kChunkBytes = BM * 128;    // one column block of a 128-row tile
-    static constexpr int kTileBytes = BM * D * 2;   // one 128 x D bf16 tile
-    static constexpr int kKStages = (D == 128) ? 3 : 4;
-    static constexpr int kVStages = (D == 128) ? 2 : 4;
+    static_assert(!F8 || D == 128, "E4M3 operands: d = 128 only");
+    static constexpr int kElemBytes = F8 ? 1 : 2;
+    static constexpr int kChunks = D * kElemBytes / 128;  // 128-byte column blocks per row
+    static constexpr int kChunkElems = 128 / kElemBytes;  // elements of a row in one column block
+    static constexpr int kChunkBytes = BM * 128;           // one column block of a 128-row tile
+    static constexpr int kTileBytes = BM * D * kElemBytes; // one 128 x D tile
+    static constexpr int kKStages = F8 ? 4 : (D == 128) ? 3 : 4;
+    static constexpr int kVStages = F8 ? 4 : (D == 128) ? 2 : 4;
     static constexpr int kOffQ = 0;                                   // Q_A, Q_B
     static constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;
@@ -124,7 +139,8 @@ struct Cfg {
     static constexpr int kBarPFull = kBarSFull + 2;          // [2]
     static constexpr int kBarOFinal = kBarPFull + 2;         // [2]
     static constexpr int kBarOFree = kBarOFinal + 2;         // [2]
-    static constexpr int kBarDrain = kBarOFree + 2;
+    static constexpr int kBarPHalf = kBarOFree + 2;          // [2] P of keys [0, 64) in TMEM
+    static constexpr int kBarDrain = kBarPHalf + 2;
     static constexpr int kNumBars = kBarDrain + 1;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 4;
@@ -282,18 +298,44 @@ __device__ __forceinline__ void exp_half(const float *s, float scale_log2, float
     lrs = ((b[0] + b[1]) + (b[2] + b[3])) + (bb.x + bb.y);
 }
 
+// E4M3 probabilities of one 128-key score row: p = 2^(s * scale_log2 - m)
+// summed unrounded into `ls` and rounded to E4M3, four keys per 32-bit
+// column (key 4c + i in byte i of column c).
+__device__ __forceinline__ void exp_e4m3(const float *s, float scale_log2, float neg_m, uint32_t (&pk)[32],
+                                         float2 &ls) {
+    const float2 sl2 = make_float2(scale_log2, scale_log2);
+    const float2 nm = make_float2(neg_m, neg_m);
+    float2 a[4] = {ls, make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int c = 0; c < 128; c += 4) {
+        const float2 x0 = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2, nm);
+        const float2 x1 = __ffma2_rn(make_float2(s[c + 2], s[c + 3]), sl2, nm);
+        const float2 p0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+        const float2 p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+        a[(c >> 2) & 3] = __fadd2_rn(a[(c >> 2) & 3], __fadd2_rn(p0, p1));
+        pk[c >> 2] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
+    }
+    ls = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+}
+
 // ------------------------------------------------------------------ softmax
 // One warpgroup, query tile x; thread owns row (warp % 4) * 32 + lane.
-template <int D, bool O_BF16>
+// E4M3 probabilities are taken relative to m_ref - kF8Shift (so that they lie
+// in (0, 2^8] with eager rescaling, inside E4M3's normal range down to 2^-14
+// of the row maximum).
+constexpr float kF8Shift = 8.f;
+
+template <int D, bool O_BF16, bool F8>
 __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
                                              uint32_t tmem, int x, int warp, int lane) {
-    using C = Cfg<D>;
+    using C = Cfg<D, F8>;
     const int row_in_tile = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float LN2 = 0.69314718055994530942f;
     const float NEG_INF = __int_as_float(0xff800000);
     uint64_t *s_full = &bars[C::kBarSFull + x];
     uint64_t *p_full = &bars[C::kBarPFull + x];
+    uint64_t *p_half = &bars[C::kBarPHalf + x];
     uint64_t *o_final = &bars[C::kBarOFinal + x];
     uint64_t *o_free = &bars[C::kBarOFree + x];
     const uint32_t t_s = tmem + lane_off + col_s(x);
@@ -375,10 +417,20 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
                     tmem_st32(t_o + ch * 32, r);
                 }
             }
-            exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
-            tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
-            exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
-            tmem_st32(t_s + 32, pk1);
+            if constexpr (F8) {
+                exp_e4m3(s, p.scale_log2, kF8Shift - m_ref, pk0, ls);
+                tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
+            } else {
+                exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
+                tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
+                if constexpr (kSplitPV<D>) {
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(p_half);
+                }
+                exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
+                tmem_st32(t_s + 32, pk1);
+            }
             l += ls.x + ls.y;
             lr += lrs;
             tmem_st_wait();
@@ -396,8 +448,12 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         tc_fence_after();
         // a row whose allowed keys all lie outside this unit's key range (key
         // splits) has nothing summed: O = 0, lse = -inf for it
-        const bool empty = !(lr > 0.f);
-        const float inv_l = empty ? 0.f : 1.f / lr;
+        // E4M3: O over the unrounded sum (with eager rescaling the row maximum's
+        // weight 2^8 is exact in E4M3, so the rounded and unrounded sums differ
+        // only by the unbiased rounding of the smaller weights)
+        const float norm = F8 ? l : lr;
+        const bool empty = !(norm > 0.f);
+        const float inv_l = empty ? 0.f : (F8 ? p.out_scale : 1.f) / norm;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
             uint32_t r[32];
@@ -406,7 +462,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             tmem_reg_fence(r);
             if (row_valid) store_row_chunk<D, O_BF16>(p.o, row_id, ch, r, inv_l);
         }
-        if (row_valid) p.lse[row_id] = empty ? NEG_INF : (m_ref + log2f(l)) * LN2;
+        if (row_valid) p.lse[row_id] = empty ? NEG_INF : (m_ref - (F8 ? kF8Shift : 0.f) + log2f(l)) * LN2;
         tc_fence_before();
         mbar_arrive(o_free);
         ++tl;
@@ -415,12 +471,12 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
 }
 
 // ------------------------------------------------------------------ MMA issuer
-template <int D>
+template <int D, bool F8>
 __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
                                          uint32_t tmem, uint32_t q_addr, uint32_t k_addr, uint32_t v_addr) {
-    using C = Cfg<D>;
-    const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-    const uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
+    using C = Cfg<D, F8>;
+    const uint32_t idesc_qk = F8 ? idesc_e4m3_f32(BM, BN, false) : idesc_bf16_f32(BM, BN, false);
+    const uint32_t idesc_pv = F8 ? idesc_e4m3_f32(BM, D, true) : idesc_bf16_f32(BM, D, true);
     // Descriptors differ only in their start-address field (bits [0,14), in
     // 16-byte units), so each operand's descriptor is a base plus an offset.
     const uint64_t q_desc = sw128_desc(q_addr, 16, 1024);
@@ -436,19 +492,38 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
     auto qk = [&](int x, uint32_t kslot) {
         const uint64_t qd = q_desc + ((x * C::kTileBytes) >> 4);
         const uint64_t kd = k_desc + ((kslot * C::kTileBytes) >> 4);
-        if constexpr (D == 128) mma_ss_k128(tmem + col_s(x), qd, kd, idesc_qk, 0u);
+        if constexpr (F8) mma_e4m3_ss_k128(tmem + col_s(x), qd, kd, idesc_qk, 0u);
+        else if constexpr (D == 128) mma_ss_k128(tmem + col_s(x), qd, kd, idesc_qk, 0u);
         else mma_ss_k64(tmem + col_s(x), qd, kd, idesc_qk, 0u);
         tc_commit(&bars[C::kBarSFull + x]);
     };
     // O_X (+)= P_X V for the value tile in ring slot vslot; `first` starts a
     // fresh accumulator, `last` ends the unit for tile X
     auto pv = [&](int x, uint32_t &gpx, uint32_t tlx, uint32_t vslot, bool first, bool last) -> bool {
-        if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
-        ++gpx;
-        if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
-        tc_fence_after();
-        mma_ts_k128(tmem + col_o(x, D), tmem + col_s(x), v_desc + ((vslot * C::kTileBytes) >> 4), idesc_pv,
-                    first ? 0u : 1u);
+        const uint64_t vd = v_desc + ((vslot * C::kTileBytes) >> 4);
+        if constexpr (F8) {
+            if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
+            ++gpx;
+            if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
+            tc_fence_after();
+            mma_e4m3_ts_k128(tmem + col_o(x, D), tmem + col_s(x), vd, idesc_pv, first ? 0u : 1u);
+        } else if constexpr (kSplitPV<D>) {
+            // keys [0, 64): P columns [0, 32), V rows [0, 64); then keys [64, 128)
+            if (!mbar_wait(&bars[C::kBarPHalf + x], gpx & 1, abort_flag, to)) return false;
+            if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
+            tc_fence_after();
+            mma_ts_k64(tmem + col_o(x, D), tmem + col_s(x), vd, idesc_pv, first ? 0u : 1u);
+            if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
+            ++gpx;
+            tc_fence_after();
+            mma_ts_k64(tmem + col_o(x, D), tmem + col_s(x) + 32, vd + (4 * 2048 >> 4), idesc_pv, 1u);
+        } else {
+            if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
+            ++gpx;
+            if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
+            tc_fence_after();
+            mma_ts_k128(tmem + col_o(x, D), tmem + col_s(x), vd, idesc_pv, first ? 0u : 1u);
+        }
         if (last) tc_commit(&bars[C::kBarOFinal + x]);
         return true;
     };
@@ -496,10 +571,10 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
 }
 
 // ------------------------------------------------------------------ TMA producer
-template <int D>
+template <int D, bool F8>
 __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
                                           uint8_t *sQ, uint8_t *sK, uint8_t *sV) {
-    using C = Cfg<D>;
+    using C = Cfg<D, F8>;
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_k);
     prefetch_tensormap(&p.tm_v);
@@ -520,8 +595,8 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
         for (int x = 0; x < kQTiles; ++x)
 #pragma unroll
             for (int c = 0; c < C::kChunks; ++c)
-                tma_load_3d(sQ + x * C::kTileBytes + c * C::kChunkBytes, &p.tm_q, &bars[C::kBarQFull], c * 64,
-                            u.blk * kUnitRows + x * BM, u.bh);
+                tma_load_3d(sQ + x * C::kTileBytes + c * C::kChunkBytes, &p.tm_q, &bars[C::kBarQFull],
+                            c * C::kChunkElems, u.blk * kUnitRows + x * BM, u.bh);
         ++tq;
         for (int j = 0; j < u.nmax && ok; ++j) {
             {
@@ -534,7 +609,7 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_3d(sK + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_k, &bars[C::kBarKFull + slot],
-                                c * 64, (u.lo + j) * BN, u.bh_kv);
+                                c * C::kChunkElems, (u.lo + j) * BN, u.bh_kv);
                 ++gk;
             }
             {
@@ -547,7 +622,7 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
                     tma_load_3d(sV + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_v, &bars[C::kBarVFull + slot],
-                                c * 64, (u.lo + j) * BN, u.bh_kv);
+                                c * C::kChunkElems, (u.lo + j) * BN, u.bh_kv);
                 ++gv;
             }
         }
@@ -567,9 +642,9 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
     }
 }
 
-template <int D, bool O_BF16>
+template <int D, bool O_BF16, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
-    using C = Cfg<D>;
+    using C = Cfg<D, F8>;
     extern __shared__ uint8_t smem_raw[];
     // 128-byte-swizzled TMA destinations and UMMA operands need 1024-byte alignment
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -585,8 +660,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
-            const bool per_row =
-                (i >= C::kBarPFull && i < C::kBarPFull + 2) || (i >= C::kBarOFree && i < C::kBarOFree + 2);
+            const bool per_row = (i >= C::kBarPFull && i < C::kBarPFull + 2) ||
+                                 (i >= C::kBarOFree && i < C::kBarOFree + 2) ||
+                                 (i >= C::kBarPHalf && i < C::kBarPHalf + 2);
             mbar_init(&bars[i], per_row ? 128u : 1u);
         }
         *abort_flag = 0;
@@ -603,19 +679,20 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
 
     if (warp < kSoftmaxWarps) {
         setmaxnreg_inc<kSoftmaxRegs>();
-        if (!softmax_role<D, O_BF16>(p, bars, abort_flag, tmem, warp >> 2, warp, lane)) record_timeout(p);
+        if (!softmax_role<D, O_BF16, F8>(p, bars, abort_flag, tmem, warp >> 2, warp, lane)) record_timeout(p);
     } else {
         setmaxnreg_dec<kControlRegs>();
     }
     if (warp == kMmaWarp) {
         if (lane == 0) {
-            if (!mma_role<D>(p, bars, abort_flag, tmem, smem_u32(sQ), smem_u32(sK), smem_u32(sV))) record_timeout(p);
+            if (!mma_role<D, F8>(p, bars, abort_flag, tmem, smem_u32(sQ), smem_u32(sK), smem_u32(sV)))
+                record_timeout(p);
             // drain: no MMA may still be running when TMEM is released
             tc_commit(&bars[C::kBarDrain]);
             mbar_wait_drain(&bars[C::kBarDrain], 0, p.timeout_ns);
         }
     } else if (warp == kLoadWarp) {
-        if (lane == 0) load_role<D>(p, bars, abort_flag, sQ, sK, sV);
+        if (lane == 0) load_role<D, F8>(p, bars, abort_flag, sQ, sK, sV);
     }
 
     tc_fence_before();

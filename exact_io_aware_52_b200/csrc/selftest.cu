@@ -4,6 +4,8 @@
 //   * S = A B^T with tcgen05.mma, both operands K-major in shared memory;
 //   * O = P V with tcgen05.mma, P packed into TMEM by tcgen05.st, V MN-major
 //     in shared memory;
+//   * the same two products with E4M3 operands (tcgen05.mma kind::f8f6f4),
+//     P rounded to E4M3 and packed four per TMEM column by the kernel's packer;
 //   * the bounded mbarrier wait running out on a barrier nobody arrives at.
 // They use exactly the descriptor builders and MMA issue blocks of the kernel.
 #include <cuda.h>
@@ -23,8 +25,9 @@ using namespace fa;
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // 1 s
 
 struct SelfParams {
-    CUtensorMap ta, tb;  // 3-D maps, box {64, 128, 1}, 128-byte swizzle
+    CUtensorMap ta, tb;  // 3-D maps, box {64, 128, 1} (bf16) or {128, 128, 1} (E4M3), 128-byte swizzle
     const uint16_t *p;   // P for the P V check, [128][128] bf16
+    const float *pf;     // P for the E4M3 P V check, [128][128] fp32 (rounded on the device)
     float *out;
     uint8_t *raw;
     int32_t *status;
@@ -201,6 +204,140 @@ __global__ void k_mma_ts(const __grid_constant__ SelfParams sp) {
 }
 
 // ---------------------------------------------------------------------------
+// S[128][128] = A[128][128] * B[128][128]^T, E4M3 operands K-major
+__global__ void k_mma_e4m3_ss(const __grid_constant__ SelfParams sp) {
+    extern __shared__ uint8_t raw_smem[];
+    uint8_t *smem = raw_smem + ((1024u - (smem_u32(raw_smem) & 1023u)) & 1023u);
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + 16384;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 32768);
+    uint32_t *slot = reinterpret_cast<uint32_t *>(smem + 32768 + 64);
+    int *abort_flag = reinterpret_cast<int *>(smem + 32768 + 68);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *slot;
+    bool ok = true;
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&bars[0], 2 * 16384);
+        tma_load_3d(sA, &sp.ta, &bars[0], 0, 0, 0);
+        tma_load_3d(sB, &sp.tb, &bars[0], 0, 0, 0);
+        ok = mbar_wait(&bars[0], 0, abort_flag, kTimeoutNs);
+        if (ok) {
+            tc_fence_after();
+            mma_e4m3_ss_k128(tmem, sw128_desc(smem_u32(sA), 16, 1024), sw128_desc(smem_u32(sB), 16, 1024),
+                             idesc_e4m3_f32(128, 128, false), 0u);
+        }
+        tc_commit(&bars[1]);
+    }
+    __syncwarp();
+    ok = mbar_wait(&bars[1], 0, abort_flag, kTimeoutNs);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+        tc_fence_after();
+        const int row = warp * 32 + lane;
+        for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + ch * 32, r);
+            tmem_ld_wait();
+            tmem_reg_fence(r);
+            for (int c = 0; c < 32; ++c) sp.out[row * 128 + ch * 32 + c] = __uint_as_float(r[c]);
+        }
+    } else {
+        set_status(sp.status, 5);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// O[128][128] = E4M3(P)[128][128] * V[128][128]: P rounded to E4M3 and packed
+// into TMEM by pack_e4m3x4, V (E4M3) MN-major in shared memory
+__global__ void k_mma_e4m3_ts(const __grid_constant__ SelfParams sp) {
+    extern __shared__ uint8_t raw_smem[];
+    uint8_t *smem = raw_smem + ((1024u - (smem_u32(raw_smem) & 1023u)) & 1023u);
+    uint8_t *sV = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 16384);
+    uint32_t *slot = reinterpret_cast<uint32_t *>(smem + 16384 + 64);
+    int *abort_flag = reinterpret_cast<int *>(smem + 16384 + 68);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *slot;
+    const uint32_t colO = 0, colP = 128;
+    const int row = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    {
+        uint32_t r[32];
+        const float *prow = sp.pf + row * 128;
+        for (int c = 0; c < 32; ++c) r[c] = pack_e4m3x4(prow[4 * c], prow[4 * c + 1], prow[4 * c + 2], prow[4 * c + 3]);
+        tmem_st32(tmem + lane_off + colP, r);
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    bool ok = true;
+    if (threadIdx.x == 0) {
+        tc_fence_after();
+        mbar_arrive_expect_tx(&bars[0], 16384);
+        tma_load_3d(sV, &sp.tb, &bars[0], 0, 0, 0);
+        ok = mbar_wait(&bars[0], 0, abort_flag, kTimeoutNs);
+        if (ok) {
+            tc_fence_after();
+            mma_e4m3_ts_k128(tmem + colO, tmem + colP, sw128_desc(smem_u32(sV), 16384, 1024),
+                             idesc_e4m3_f32(128, 128, true), 0u);
+        }
+        tc_commit(&bars[1]);
+    }
+    __syncwarp();
+    ok = mbar_wait(&bars[1], 0, abort_flag, kTimeoutNs);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+        tc_fence_after();
+        for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(tmem + lane_off + colO + ch * 32, r);
+            tmem_ld_wait();
+            tmem_reg_fence(r);
+            for (int c = 0; c < 32; ++c) sp.out[row * 128 + ch * 32 + c] = __uint_as_float(r[c]);
+        }
+    } else {
+        set_status(sp.status, 5);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // A wait on a barrier that nothing ever arrives at must give up after the
 // limit and report it, leaving the context usable.
 __global__ void k_wait_timeout(int32_t *status, uint64_t timeout_ns) {
@@ -245,6 +382,21 @@ int make_map(CUtensorMap *m, const void *base, int rows, int cols) {
     cuuint32_t box[3] = {64, 128, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+               ? 0
+               : 4;
+}
+
+// 3-D map over a [rows][128] byte tensor (E4M3), box {128, 128, 1}, 128-byte swizzle
+int make_map8(CUtensorMap *m, const void *base, int rows) {
+    auto enc = encoder();
+    if (!enc) return 4;
+    cuuint64_t dims[3] = {128, (cuuint64_t)rows, 1};
+    cuuint64_t strides[2] = {128, (cuuint64_t)rows * 128};
+    cuuint32_t box[3] = {128, 128, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
                ? 0
@@ -296,6 +448,33 @@ int fa_selftest_mma_ts(const void *p, const void *v, float *o, int D, int32_t *s
     const int smem = 32768 + 128 + 1024;
     if (cudaFuncSetAttribute(k_mma_ts, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 4;
     k_mma_ts<<<1, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(sp);
+    return finish(stream);
+}
+
+int fa_selftest_mma_e4m3_ss(const void *a, const void *b, float *s, int32_t *status, void *stream) {
+    SelfParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    if (make_map8(&sp.ta, a, 128) || make_map8(&sp.tb, b, 128)) return 4;
+    sp.out = s;
+    sp.status = status;
+    const int smem = 32768 + 128 + 1024;
+    if (cudaFuncSetAttribute(k_mma_e4m3_ss, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return 4;
+    k_mma_e4m3_ss<<<1, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(sp);
+    return finish(stream);
+}
+
+int fa_selftest_mma_e4m3_ts(const float *p, const void *v, float *o, int32_t *status, void *stream) {
+    SelfParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    if (make_map8(&sp.tb, v, 128)) return 4;
+    sp.pf = p;
+    sp.out = o;
+    sp.status = status;
+    const int smem = 16384 + 128 + 1024;
+    if (cudaFuncSetAttribute(k_mma_e4m3_ts, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return 4;
+    k_mma_e4m3_ts<<<1, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(sp);
     return finish(stream);
 }
 

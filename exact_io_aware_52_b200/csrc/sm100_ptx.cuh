@@ -309,7 +309,80 @@ __device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, ui
         "}" ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// O (+)= P V over 64 keys (4 steps of K = 16): a_tmem and b_desc point at the
+// first of the 64 keys (P column a_tmem, V key row b_desc).
+__device__ __forceinline__ void mma_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t.reg .pred p, pt;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 pt, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        FA_TS_STEP(8, 128) FA_TS_STEP(16, 256) FA_TS_STEP(24, 384)
+        "}" ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 #undef FA_TS_STEP
+
+// ---------------------------------------------------------------- 8-bit operands
+// Instruction descriptor of tcgen05.mma kind::f8f6f4 with both operands E4M3
+// (format code 0) and fp32 accumulation: as idesc_bf16_f32 with the A and B
+// format fields left at 0.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool b_mn_major) {
+    return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// S (+)= A B^T over K = 128 E4M3 elements: both operands K-major, 128-byte
+// rows (one 128-element row per swizzle row), 4 steps of K = 32 = 32 bytes.
+#define FA_F8SS_STEP(OFF)                                    \
+    "add.s64 da, %1, " #OFF ";\n\t"                          \
+    "add.s64 db, %2, " #OFF ";\n\t"                          \
+    "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %3, pt;\n\t"
+__device__ __forceinline__ void mma_e4m3_ss_k128(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 da, db;\n\t.reg .pred p, pt;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 pt, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t"
+        FA_F8SS_STEP(2) FA_F8SS_STEP(4) FA_F8SS_STEP(6)
+        "}" ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+#undef FA_F8SS_STEP
+
+// O (+)= P V over 128 keys of E4M3: P in TMEM (four keys per 32-bit column,
+// 8 columns per step of K = 32), V MN-major in shared memory, 32 key rows of
+// 128 bytes per step (4096 bytes = 256 in 16-byte units).
+#define FA_F8TS_STEP(TA, DB)                                 \
+    "add.u32 ta, %1, " #TA ";\n\t"                           \
+    "add.s64 db, %2, " #DB ";\n\t"                           \
+    "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [ta], db, %3, pt;\n\t"
+__device__ __forceinline__ void mma_e4m3_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t.reg .pred p, pt;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 pt, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t"
+        FA_F8TS_STEP(8, 256) FA_F8TS_STEP(16, 512) FA_F8TS_STEP(24, 768)
+        "}" ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+#undef FA_F8TS_STEP
+
+// Four fp32 values rounded to E4M3 (nearest even, saturating) and packed into
+// one 32-bit word, a in the lowest byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r)
+        : "f"(a), "f"(b), "f"(c), "f"(d));
+    return r;
+}
 
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -34,6 +34,7 @@ class Workload:
     H_kv: int | None = None            # key/value heads (grouped attention); None: H
     Nk: int | None = None              # keys (more keys than queries: cached keys); None: N
     splits: int = 0                    # key splits the benchmark uses (0: none, -1: library's choice)
+    dtype: str = "bf16"                # element type of Q, K, V: "bf16" or "e4m3"
     seed: int = 0
     notes: str = field(default="", compare=False)
 
@@ -80,22 +81,27 @@ WORKLOADS = {
     # head dimension 256: the FLOPs of workload 4 with half the heads
     8: Workload("long-context causal B1 H16 N16384 d256", 1, 16, 16384, 256, True,
                 sample_rows_per_head=256, seed=52008),
+    # FP8: the shape of workload 4 with E4M3 inputs (unit scales)
+    9: Workload("long-context causal FP8-E4M3 B1 H32 N16384 d128", 1, 32, 16384, 128, True,
+                sample_rows_per_head=64, seed=52009, dtype="e4m3"),
 }
 
 
 def make_inputs(w: Workload, seed: int | None = None):
     """Draw (q, k, v, k_len) on the CPU for workload ``w``.
 
-    q: bfloat16 [B, H, N, d]; k, v: bfloat16 [B, H_kv, N_k, d] contiguous CPU tensors.
+    q: [B, H, N, d]; k, v: [B, H_kv, N_k, d] contiguous CPU tensors of bfloat16
+    (or float8_e4m3fn, rounded from the same float32 draws, for dtype "e4m3").
     k_len: int32 [B] CPU tensor, or None when the workload has no key padding.
     """
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed if seed is None else seed)
     shape = (w.B, w.H, w.N, w.d)
     kv_shape = (w.B, w.kv_heads, w.keys, w.d)
-    q = (torch.randn(shape, generator=g, dtype=torch.float32) * w.qk_std).to(torch.bfloat16)
-    k = (torch.randn(kv_shape, generator=g, dtype=torch.float32) * w.qk_std).to(torch.bfloat16)
-    v = torch.randn(kv_shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    dt = torch.float8_e4m3fn if w.dtype == "e4m3" else torch.bfloat16
+    q = (torch.randn(shape, generator=g, dtype=torch.float32) * w.qk_std).to(dt)
+    k = (torch.randn(kv_shape, generator=g, dtype=torch.float32) * w.qk_std).to(dt)
+    v = torch.randn(kv_shape, generator=g, dtype=torch.float32).to(dt)
     k_len = None
     if w.kpad is not None:
         lo, hi = w.kpad
@@ -125,7 +131,7 @@ def sample_rows(w: Workload, seed: int | None = None):
 
 
 def custom(B, H, N, d, causal, qk_std=1.0, kpad=None, seed=1, name="custom", H_kv=None, Nk=None,
-           splits=0) -> Workload:
+           splits=0, dtype="bf16") -> Workload:
     """A workload of arbitrary shape (tests of ragged and edge shapes)."""
     return Workload(name, B, H, N, d, causal, qk_std=qk_std, kpad=kpad, seed=seed, H_kv=H_kv, Nk=Nk,
-                    splits=splits)
+                    splits=splits, dtype=dtype)

@@ -68,6 +68,12 @@ typedef enum {
 
 typedef enum { FA_O_F32 = 0, FA_O_BF16 = 1 } fa_o_dtype;
 
+/* Element type of q, k and v. */
+typedef enum {
+    FA_IN_BF16 = 0, /* bfloat16, the default                                        */
+    FA_IN_E4M3 = 1  /* FP8 E4M3 (one byte; OCP "fn" variant: no infinities), d = 128 */
+} fa_in_dtype;
+
 /* Flags for fa_fwd_params.flags. */
 enum {
     /* Rescale the running output whenever a row maximum grows, instead of
@@ -94,7 +100,7 @@ FA_EXPORT fa_status fa_fwd(const void *q, const void *k, const void *v, float *o
                  int B, int H, int N, int d, int causal, float scale, void *stream);
 
 typedef struct {
-    const void *q, *k, *v;   /* device bf16: q [B, H, N, d]; k, v [B, H_kv, N, d]     */
+    const void *q, *k, *v;   /* device, in_dtype: q [B, H, N, d]; k, v [B, H_kv, N_k, d] */
     void *o;                 /* device [B, H, N, d], fp32 or bf16 per o_dtype         */
     float *lse;              /* device fp32 [B, H, N]                                 */
     const int32_t *k_len;    /* device int32 [B], or NULL (no key padding)           */
@@ -121,6 +127,13 @@ typedef struct {
                                 num_splits <= 1.  Owned by the caller; the library
                                 writes every byte it reads from it in the same call   */
     size_t workspace_bytes;  /* size of workspace                                     */
+    int in_dtype;            /* fa_in_dtype of q, k, v                                */
+    float descale_q, descale_k, descale_v;
+                             /* E4M3 inputs: the values are q * descale_q, k * descale_k,
+                                v * descale_v (per-tensor scales; 0 means 1).  Ignored
+                                for bf16.  The products Q K^T and P V run on E4M3 with
+                                fp32 accumulation; P is rounded to E4M3 before P V;
+                                the softmax is fp32.  Finite and >= 0.                */
 } fa_fwd_params;
 
 /*
@@ -149,7 +162,7 @@ FA_EXPORT int fa_fwd_suggest_splits(const fa_fwd_params *p);
 FA_EXPORT fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream);
 
 typedef struct {
-    const void *q, *k, *v;   /* host bf16, shapes as in dev (pinned for async copies) */
+    const void *q, *k, *v;   /* host, dev.in_dtype, shapes as in dev (pinned for async copies) */
     const int32_t *k_len;    /* host int32 [B] or NULL                                */
     void *o;                 /* host output, dtype per dev.o_dtype                    */
     float *lse;              /* host fp32 [B, H, N]                                   */

@@ -40,6 +40,17 @@ FA_SELFTEST_EXPORT int fa_selftest_mma_ss(const void *a, const void *b, float *s
 FA_SELFTEST_EXPORT int fa_selftest_mma_ts(const void *p, const void *v, float *o, int D, int32_t *status,
                                           void *stream);
 
+/* s[128][128] (fp32) = a[128][128] * b[128][128]^T with tcgen05.mma
+ * kind::f8f6f4, a and b E4M3 (one byte each) K-major in shared memory. */
+FA_SELFTEST_EXPORT int fa_selftest_mma_e4m3_ss(const void *a, const void *b, float *s, int32_t *status,
+                                               void *stream);
+
+/* o[128][128] (fp32) = E4M3(p)[128][128] * v[128][128]: p given in fp32 is
+ * rounded to E4M3 (nearest even, saturating) and packed four per TMEM column
+ * by the kernel's packer; v E4M3 MN-major in shared memory. */
+FA_SELFTEST_EXPORT int fa_selftest_mma_e4m3_ts(const float *p, const void *v, float *o, int32_t *status,
+                                               void *stream);
+
 /* y[i] = 2^x[i] (fp32, n even) through the FMA-pipe polynomial exponential the
  * kernel uses for part of its softmax weights (the online softmax of section
  * "Calculo de Softmax en linea"); inputs below -127 give +0. */

@@ -15,7 +15,8 @@ TOL_MEAN = 1e-3   # mean |O_gpu - O_ref|
 TOL_LSE = 1e-4    # max |lse_gpu - lse_ref| / max(|lse_ref|, 1)
 
 
-def run_gpu(q, k, v, causal, scale, k_len=None, out_dtype=torch.float32, flags=0, stream=None, num_splits=0):
+def run_gpu(q, k, v, causal, scale, k_len=None, out_dtype=torch.float32, flags=0, stream=None, num_splits=0,
+            descale=(0.0, 0.0, 0.0)):
     """Run fa_fwd_ex on cuda:0; returns (O [B,H,N,d] fp32 CPU, lse [B,H,N] CPU).
 
     Outputs (and any split workspace) start as NaN so rows the kernels fail to
@@ -34,7 +35,7 @@ def run_gpu(q, k, v, causal, scale, k_len=None, out_dtype=torch.float32, flags=0
         nbytes = fb.workspace_bytes(qd, kd, num_splits)
         ws = torch.full((max(nbytes, 16) // 4,), float("nan"), dtype=torch.float32, device=dev)
     fb.fa_fwd_ex(qd, kd, vd, o, lse, causal, scale, k_len=kl, dev_status=status, flags=flags, stream=stream,
-                 num_splits=num_splits, workspace=ws)
+                 num_splits=num_splits, workspace=ws, descale=descale)
     st = fb.read_device_status(status, stream=stream)
     assert st == fb.FA_OK, fb.status_string(st)
     return o.float().cpu(), lse.cpu()

@@ -43,13 +43,14 @@ def test_status_strings_and_version():
     for code, name in names.items():
         assert fb.status_string(code) == name
     assert fb.status_string(99) == "FA_ERR_UNKNOWN"
-    assert fb.version() == 200
+    assert fb.version() == 300
 
 
 def _params(**kw):
     base = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0x50000, k_len=None, dev_status=None,
                 B=1, H=2, N=128, d=64, causal=0, scale=0.125, o_dtype=0, flags=0, timeout_ms=0, H_kv=0,
-                N_k=0, num_splits=0, workspace=None, workspace_bytes=0)
+                N_k=0, num_splits=0, workspace=None, workspace_bytes=0, in_dtype=0, descale_q=0.0, descale_k=0.0,
+                descale_v=0.0)
     base.update(kw)
     return fb.FaParams(**base)
 
@@ -85,6 +86,12 @@ def _ex(**kw):
     (dict(N_k=1024, num_splits=4, workspace=0x80000, workspace_bytes=64), fb.FA_ERR_INVALID_ARGUMENT),
     (dict(N_k=1024, num_splits=4, workspace=0x80008, workspace_bytes=1 << 30), fb.FA_ERR_MISALIGNED),
     (dict(d=32), fb.FA_ERR_UNSUPPORTED),
+    (dict(in_dtype=2), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(in_dtype=1, descale_q=-1.0), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(in_dtype=1, descale_v=float("nan")), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(descale_k=float("inf")), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(in_dtype=1, d=64), fb.FA_ERR_UNSUPPORTED),               # E4M3 inputs: d = 128 only
+    (dict(in_dtype=1, d=256), fb.FA_ERR_UNSUPPORTED),
     (dict(d=512), fb.FA_ERR_UNSUPPORTED),
     (dict(d=192), fb.FA_ERR_UNSUPPORTED),
     (dict(d=96), fb.FA_ERR_UNSUPPORTED),

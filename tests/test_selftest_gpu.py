@@ -75,6 +75,37 @@ def test_tcgen05_ts_matches_matmul(D):
     np.testing.assert_allclose(o.cpu().double().numpy(), ref.numpy(), rtol=0, atol=2e-4)
 
 
+def test_tcgen05_e4m3_ss_matches_matmul():
+    """S = A B^T with E4M3 operands (kind::f8f6f4, K-major, 128-byte rows)
+    equals the float64 product of the same E4M3 values."""
+    lib = fb.load_selftest()
+    g = torch.Generator().manual_seed(300)
+    a = (torch.randn(128, 128, generator=g) * 3).to(torch.float8_e4m3fn)
+    b = (torch.randn(128, 128, generator=g) * 3).to(torch.float8_e4m3fn)
+    s = torch.full((128, 128), float("nan"), device=_dev())
+    st = _status()
+    assert lib.fa_selftest_mma_e4m3_ss(_p(a.to(_dev())), _p(b.to(_dev())), _p(s), _p(st), None) == 0
+    assert st.item() == 0
+    ref = a.double() @ b.double().T
+    np.testing.assert_allclose(s.cpu().double().numpy(), ref.numpy(), rtol=1e-6, atol=1e-4)
+
+
+def test_tcgen05_e4m3_ts_matches_matmul():
+    """O = E4M3(P) V: P (fp32, spanning the E4M3 subnormals up to 256) rounded
+    and packed four per TMEM column by the kernel's packer, V MN-major; equals
+    the float64 product of torch's E4M3 rounding of P with V."""
+    lib = fb.load_selftest()
+    g = torch.Generator().manual_seed(301)
+    p = torch.exp2(torch.rand(128, 128, generator=g) * 22 - 14)  # 2^-14 .. 2^8
+    v = torch.randn(128, 128, generator=g).to(torch.float8_e4m3fn)
+    o = torch.full((128, 128), float("nan"), device=_dev())
+    st = _status()
+    assert lib.fa_selftest_mma_e4m3_ts(_p(p.to(_dev())), _p(v.to(_dev())), _p(o), _p(st), None) == 0
+    assert st.item() == 0
+    ref = p.to(torch.float8_e4m3fn).double() @ v.double()
+    np.testing.assert_allclose(o.cpu().double().numpy(), ref.numpy(), rtol=1e-5, atol=1e-4)
+
+
 def test_bounded_wait_gives_up():
     """A wait on a barrier nothing arrives at gives up after its limit,
     reports FA_ERR_DEVICE_TIMEOUT, and the context stays usable."""

@@ -58,6 +58,19 @@ class FaHostParams(ctypes.Structure):
     ]
 
 
+class FaBwdParams(ctypes.Structure):
+    """Mirror of fa_bwd_params (include/fa.h)."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("o", ctypes.c_void_p),
+        ("dout", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p),
+        ("dv", ctypes.c_void_p), ("k_len", ctypes.c_void_p), ("dev_status", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int),
+        ("causal", ctypes.c_int), ("scale", ctypes.c_float), ("o_dtype", ctypes.c_int),
+        ("timeout_ms", ctypes.c_uint32), ("H_kv", ctypes.c_int), ("N_k", ctypes.c_int),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 class FaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -90,6 +103,10 @@ def load():
             lib.fa_fwd_workspace_bytes.argtypes = [ctypes.POINTER(FaParams)]
             lib.fa_fwd_suggest_splits.restype = i
             lib.fa_fwd_suggest_splits.argtypes = [ctypes.POINTER(FaParams)]
+            lib.fa_bwd.restype = i
+            lib.fa_bwd.argtypes = [ctypes.POINTER(FaBwdParams), ctypes.c_void_p]
+            lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+            lib.fa_bwd_workspace_bytes.argtypes = [ctypes.POINTER(FaBwdParams)]
             lib.fa_fwd_static_workspace.restype = i
             lib.fa_fwd_static_workspace.argtypes = [ctypes.POINTER(FaParams), ctypes.c_void_p]
             _lib = lib
@@ -254,3 +271,45 @@ def attention(q, k, v, causal: bool, scale: float, k_len=None, out_dtype=None, f
     fa_fwd_ex(q, k, v, o, lse, causal, scale, k_len=k_len, flags=flags, stream=stream, num_splits=num_splits,
               workspace=ws, descale=descale)
     return o, lse
+
+
+def make_bwd_params(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, k_len=None, dev_status=None, timeout_ms=0,
+                    workspace=None, shape=None) -> FaBwdParams:
+    """Fill a fa_bwd_params from tensors (q, dout, o, dq [B, H, N, d]; k, v, dk, dv
+    [B, H_kv, N_k, d]; lse [B, H, N])."""
+    import torch
+    if shape is None:
+        shape = tuple(q.shape)
+    B, H, N, d = shape
+    kv4 = k is not None and hasattr(k, "shape") and k.dim() == 4
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return FaBwdParams(q=_ptr(q), k=_ptr(k), v=_ptr(v), o=_ptr(o), dout=_ptr(dout), lse=_ptr(lse), dq=_ptr(dq),
+                       dk=_ptr(dk), dv=_ptr(dv), k_len=_ptr(k_len), dev_status=_ptr(dev_status), B=B, H=H, N=N,
+                       d=d, causal=int(bool(causal)), scale=float(scale),
+                       o_dtype=FA_O_BF16 if (o is not None and o.dtype == torch.bfloat16) else FA_O_F32,
+                       timeout_ms=int(timeout_ms), H_kv=int(k.shape[1]) if kv4 else 0,
+                       N_k=int(k.shape[2]) if kv4 else 0, workspace=_ptr(workspace), workspace_bytes=ws_bytes)
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal: bool, scale: float, workspace, k_len=None, dev_status=None,
+           timeout_ms: int = 0, stream=None):
+    """fa_bwd: gradients dq, dk, dv (fp32 CUDA tensors, overwritten) of the forward
+    (o, lse) for dout; workspace: CUDA tensor of >= fa_bwd_workspace_bytes bytes."""
+    p = make_bwd_params(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, k_len, dev_status, timeout_ms, workspace)
+    _check(load().fa_bwd(ctypes.byref(p), _stream(stream)), "fa_bwd")
+
+
+def bwd_workspace_bytes(q) -> int:
+    B, H, N, _ = q.shape
+    return 4 * B * H * N
+
+
+def attention_bwd(q, k, v, o, lse, dout, causal: bool, scale: float, k_len=None, stream=None):
+    """Allocate dq, dk, dv (fp32) and the workspace with torch on q's device and run fa_bwd."""
+    import torch
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    ws = torch.empty(max(bwd_workspace_bytes(q), 16), dtype=torch.uint8, device=q.device)
+    fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, causal, scale, ws, k_len=k_len, stream=stream)
+    return dq, dk, dv

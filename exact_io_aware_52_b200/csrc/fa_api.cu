@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_bwd_kernel.cuh"
 #include "fa_combine_kernel.cuh"
 #include "fa_fwd_d256_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
@@ -26,6 +27,7 @@ struct DeviceInfo {
     bool supported = false;
     int num_sms = 0;
     bool attr_set[4][2] = {};  // [d = 64, 128, 256, 128 with E4M3 inputs][bf16 out]
+    bool bwd_attr_set[2] = {};  // backward kernel, [d == 128]
 };
 
 std::mutex g_mu;
@@ -189,9 +191,113 @@ fa_status launch_combine_d(int d, const float *o_part, const float *lse_part, vo
     return launch_combine<256, BF16>(o_part, lse_part, o, lse, splits, rows, num_sms, stream);
 }
 
+fa_status validate_bwd(const fa_bwd_params *p) {
+    if (!p) return FA_ERR_INVALID_ARGUMENT;
+    if (p->B < 0 || p->H < 0 || p->N < 0 || p->N_k < 0) return FA_ERR_INVALID_ARGUMENT;
+    if (!(std::isfinite(p->scale) && p->scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
+    if (p->causal != 0 && p->causal != 1) return FA_ERR_INVALID_ARGUMENT;
+    if (p->o_dtype != FA_O_F32 && p->o_dtype != FA_O_BF16) return FA_ERR_INVALID_ARGUMENT;
+    if (p->H_kv < 0 || (p->H_kv > 0 && p->H % p->H_kv != 0)) return FA_ERR_INVALID_ARGUMENT;
+    if (p->d != 64 && p->d != 128) return FA_ERR_UNSUPPORTED;
+    const long long rows = (long long)p->B * p->H * p->N;
+    if (rows == 0) return FA_OK;
+    const int H_kv = p->H_kv > 0 ? p->H_kv : p->H;
+    const int n_k = p->N_k > 0 ? p->N_k : p->N;
+    if ((long long)p->B * H_kv * ((n_k + 127) / 128) > 0x7fffffffLL || (long long)p->B * p->H > 0x7fffffffLL)
+        return FA_ERR_INVALID_ARGUMENT;
+    if (!p->q || !p->k || !p->v || !p->o || !p->dout || !p->lse || !p->dq || !p->dk || !p->dv)
+        return FA_ERR_INVALID_ARGUMENT;
+    if (!p->workspace || p->workspace_bytes < (size_t)rows * sizeof(float)) return FA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v) || !aligned16(p->o) || !aligned16(p->dout) ||
+        !aligned16(p->dq) || !aligned16(p->dk) || !aligned16(p->dv) || !aligned16(p->workspace) ||
+        !aligned16(p->lse))
+        return FA_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(p->k_len) & 3u) || (reinterpret_cast<uintptr_t>(p->dev_status) & 3u))
+        return FA_ERR_MISALIGNED;
+    return FA_OK;
+}
+
+template <int D>
+fa_status launch_bwd(const fa::bwd::BwdParams &kp, const fa_bwd_params *p, DeviceInfo &di, cudaStream_t s) {
+    const long long rows = (long long)p->B * p->H * p->N;
+    long long blocks = (rows * 32 + 255) / 256;
+    if (blocks > 8LL * di.num_sms) blocks = 8LL * di.num_sms;
+    if (p->o_dtype == FA_O_BF16)
+        fa::fa_bwd_prep_kernel<D, true><<<(int)blocks, 256, 0, s>>>(
+            p->o, static_cast<const uint16_t *>(p->dout), static_cast<float *>(p->workspace), p->dq, rows);
+    else
+        fa::fa_bwd_prep_kernel<D, false><<<(int)blocks, 256, 0, s>>>(
+            p->o, static_cast<const uint16_t *>(p->dout), static_cast<float *>(p->workspace), p->dq, rows);
+    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
+    auto kern = fa::fa_bwd_sm100_kernel<D>;
+    const int smem = fa::bwd::BCfg<D>::kSmemBytes;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        bool &set = di.bwd_attr_set[D == 128];
+        if (!set) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+                return FA_ERR_CUDA;
+            set = true;
+        }
+    }
+    const int grid = kp.n_units < di.num_sms ? kp.n_units : di.num_sms;
+    kern<<<grid, fa::bwd::kThreads, smem, s>>>(kp);
+    return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t fa_bwd_workspace_bytes(const fa_bwd_params *p) {
+    if (!p || p->B <= 0 || p->H <= 0 || p->N <= 0) return 0;
+    return (size_t)p->B * p->H * p->N * sizeof(float);
+}
+
+fa_status fa_bwd(const fa_bwd_params *p, void *stream) {
+    fa_status st = validate_bwd(p);
+    if (st != FA_OK) return st;
+    if ((long long)p->B * p->H * p->N == 0) return FA_OK;
+    int dev = 0;
+    DeviceInfo *di = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        st = probe_device(&dev, &di);
+        if (st == FA_OK) st = load_encoder();
+    }
+    if (st != FA_OK) return st;
+    fa::bwd::BwdParams kp;
+    std::memset(&kp, 0, sizeof kp);
+    const int BH = p->B * p->H;
+    const int H_kv = p->H_kv > 0 ? p->H_kv : p->H;
+    const int n_k = p->N_k > 0 ? p->N_k : p->N;
+    if ((st = encode_map(&kp.tm_q, p->q, BH, p->N, p->d)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_do, p->dout, BH, p->N, p->d)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_k, p->k, p->B * H_kv, n_k, p->d)) != FA_OK) return st;
+    if ((st = encode_map(&kp.tm_v, p->v, p->B * H_kv, n_k, p->d)) != FA_OK) return st;
+    kp.lse = p->lse;
+    kp.delta = static_cast<const float *>(p->workspace);
+    kp.dq = p->dq;
+    kp.dk = p->dk;
+    kp.dv = p->dv;
+    kp.k_len = p->k_len;
+    kp.status = p->dev_status;
+    kp.B = p->B;
+    kp.H = p->H;
+    kp.N = p->N;
+    kp.Nk = n_k;
+    kp.H_kv = H_kv;
+    kp.group = p->H / H_kv;
+    kp.n_kv_tiles = (n_k + fa::BN - 1) / fa::BN;
+    kp.n_units = p->B * H_kv * kp.n_kv_tiles;
+    kp.causal = p->causal;
+    kp.scale = p->scale;
+    kp.scale_log2 = (float)((double)p->scale * 1.4426950408889634074);
+    kp.timeout_ns = (uint64_t)(p->timeout_ms ? p->timeout_ms : 2000u) * 1000000ull;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return p->d == 64 ? launch_bwd<64>(kp, p, *di, s) : launch_bwd<128>(kp, p, *di, s);
+}
+
 
 fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     fa_status st = validate(p);

@@ -309,6 +309,32 @@ __device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, ui
         "}" ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D (+)= A B over K = 128 with both operands MN-major in shared memory (A's
+// rows and B's columns contiguous, 128-byte swizzle): 8 steps of K = 16, each
+// 16 K-rows of 128 bytes (2048 bytes = 128 in 16-byte units) into both.
+#define FA_SSMN_STEP(OFF)                                    \
+    "add.s64 da, %1, " #OFF ";\n\t"                          \
+    "add.s64 db, %2, " #OFF ";\n\t"                          \
+    "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, pt;\n\t"
+__device__ __forceinline__ void mma_ss_mn_k128(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 da, db;\n\t.reg .pred p, pt;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 pt, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        FA_SSMN_STEP(128) FA_SSMN_STEP(256) FA_SSMN_STEP(384) FA_SSMN_STEP(512)
+        FA_SSMN_STEP(640) FA_SSMN_STEP(768) FA_SSMN_STEP(896)
+        "}" ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+#undef FA_SSMN_STEP
+
+// bf16 x bf16 -> fp32 instruction descriptor with a chosen major-ness of A.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return idesc_bf16_f32(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
 // O (+)= P V over 64 keys (4 steps of K = 16): a_tmem and b_desc point at the
 // first of the 64 keys (P column a_tmem, V key row b_desc).
 __device__ __forceinline__ void mma_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,

@@ -191,6 +191,50 @@ FA_EXPORT const char *fa_status_string(fa_status s);
 /* Library version as an integer MAJOR*10000 + MINOR*100 + PATCH. */
 FA_EXPORT int fa_version(void);
 
+/*
+ * Backward pass: the gradients of the forward's O with respect to q, k and v
+ * for a given dO.  The pages report training speed-ups of the method (page
+ * "FlashAttention (ES)", section "Impacto en el rendimiento") but give no
+ * backward algorithm; this is the derivative of the definition of section
+ * "El problema de la atencion estandar", with P recomputed from q, k and the
+ * forward's lse:
+ *     dV = P^T dO,  dP = dO V^T,  dS = scale * P o (dP - D),  D_i = dO_i . O_i,
+ *     dQ = dS K,    dK = dS^T Q
+ * (o the elementwise product).  Masks, N_k, grouped heads and k_len are those
+ * of the forward; dK and dV of a key/value head sum over its query heads.
+ */
+typedef struct {
+    const void *q, *k, *v;   /* device bf16: q [B, H, N, d]; k, v [B, H_kv, N_k, d]    */
+    const void *o;           /* device forward output [B, H, N, d], fp32 or bf16 (o_dtype) */
+    const void *dout;        /* device bf16 [B, H, N, d]: gradient of the loss w.r.t. O  */
+    const float *lse;        /* device fp32 [B, H, N] from the forward with the same inputs */
+    float *dq;               /* device fp32 [B, H, N, d], overwritten                   */
+    float *dk, *dv;          /* device fp32 [B, H_kv, N_k, d], overwritten              */
+    const int32_t *k_len;    /* device int32 [B] or NULL, as in fa_fwd_params           */
+    int32_t *dev_status;     /* device status word or NULL, as in fa_fwd_params         */
+    int B, H, N, d;          /* d in {64, 128}                                          */
+    int causal;
+    float scale;
+    int o_dtype;             /* fa_o_dtype of o                                         */
+    uint32_t timeout_ms;     /* per-wait time limit on the device; 0 = 2000 ms          */
+    int H_kv, N_k;           /* 0 means H and N                                         */
+    void *workspace;         /* device scratch of at least fa_bwd_workspace_bytes(p),
+                                16-byte aligned, owned by the caller                    */
+    size_t workspace_bytes;
+} fa_bwd_params;
+
+/* Scratch bytes fa_bwd needs for *p: D, fp32 [B, H, N].  0 for a NULL p. */
+FA_EXPORT size_t fa_bwd_workspace_bytes(const fa_bwd_params *p);
+
+/*
+ * fa_bwd -- two launches on `stream`: D and a zeroed dQ, then the gradients
+ * (dQ accumulated in fp32 with atomic adds, one key tile per work unit).
+ * All pointers except k_len and dev_status must be 16-byte aligned.  Errors
+ * as for fa_fwd_ex (d not in {64, 128}: FA_ERR_UNSUPPORTED).  dq, dk and dv
+ * are deterministic up to the order of the fp32 additions into dq.
+ */
+FA_EXPORT fa_status fa_bwd(const fa_bwd_params *p, void *stream);
+
 /* Size of the library's fixed device scratch array (64 MiB), per device. */
 #define FA_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
 

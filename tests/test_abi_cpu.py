@@ -163,3 +163,36 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(fb, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         fb.load()
+
+
+def _bwd_params(**kw):
+    base = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, dout=0x50000, lse=0x60000, dq=0x70000, dk=0x80000,
+                dv=0x90000, k_len=None, dev_status=None, B=1, H=2, N=128, d=64, causal=0, scale=0.125, o_dtype=0,
+                timeout_ms=0, H_kv=0, N_k=0, workspace=0xA0000, workspace_bytes=1 << 20)
+    base.update(kw)
+    return fb.FaBwdParams(**base)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(dout=None), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(dq=None), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(workspace=None), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(workspace_bytes=100), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(scale=0.0), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(causal=3), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(H_kv=3), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(N_k=-1), fb.FA_ERR_INVALID_ARGUMENT),
+    (dict(d=256), fb.FA_ERR_UNSUPPORTED),
+    (dict(dq=0x70008), fb.FA_ERR_MISALIGNED),
+    (dict(workspace=0xA0004), fb.FA_ERR_MISALIGNED),
+    (dict(B=0, q=None), fb.FA_OK),
+])
+def test_bwd_argument_errors_are_synchronous(kw, expect):
+    assert fb.load().fa_bwd(ctypes.byref(_bwd_params(**kw)), None) == expect
+
+
+def test_bwd_workspace_bytes():
+    lib = fb.load()
+    assert lib.fa_bwd_workspace_bytes(ctypes.byref(_bwd_params(B=2, H=3, N=100))) == 2 * 3 * 100 * 4
+    assert lib.fa_bwd_workspace_bytes(None) == 0

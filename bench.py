@@ -193,7 +193,8 @@ def dist_setup(args):
 def workload_config(w, world: int, q_bytes: int) -> dict:
     """The `config` object of the JSON line (identical for both arms)."""
     return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "N": w.N, "N_k": w.keys, "d": w.d,
-            "causal": w.causal, "key_splits": w.splits, "out": "fp32 O + fp32 lse",
+            "causal": w.causal, "key_splits": w.splits, "pass": w.pass_,
+            "out": "fp32 O + fp32 lse" if w.pass_ == "fwd" else "fp32 dQ, dK, dV",
             "flops_per_step_per_gpu": w.flops(),
             "l2": "inputs larger than L2 (Q,K,V %.0f MB > 126 MB); no flush" % (q_bytes / 1e6),
             "parallelism": f"replicas x{world}"}
@@ -258,11 +259,30 @@ def cpu_oracle_rate(w, q, k, v, k_len, budget_s: float, seed: int = 0):
     return flops / dt / 1e12, threads, desc, dt
 
 
+def bwd_oracle_sample(w, q, k, v, do, threads: int):
+    """A bounded sample of a backward workload for the fp64 backward oracle:
+    the first min(H, threads) query heads (with their key/value heads) and the
+    first 1024 queries and keys; returns (callable, its FLOPs, description)."""
+    import oracle
+    n = min(w.N, 1024)
+    hs = max(1, min(w.H, threads) // max(1, w.H // w.kv_heads) * max(1, w.H // w.kv_heads))
+    hk = max(1, hs // max(1, w.H // w.kv_heads))
+    sub = workloads.custom(1, hs, n, w.d, w.causal, H_kv=hk)
+    qs, ks, vs, ds = (t[:1, :h, :n].contiguous() for t, h in ((q, hs), (k, hk), (v, hk), (do, hs)))
+    flops = sub.flops() * 2.5
+
+    def run():
+        oracle.attention_bwd_f64(qs, ks, vs, ds, w.causal, w.scale, nthreads=threads)
+    return run, flops, f"backward of the first {hs} heads x {n} queries and keys (fp64 oracle)"
+
+
 def run_reference(args, world, rank):
     """The reference arm: the fp64 CPU oracle, bounded sample per step."""
     w = workloads.WORKLOADS[args.workload]
     if rank != 0:
         return  # rank 0 alone times the oracle
+    if w.pass_ == "bwd":
+        return run_reference_bwd(args, world, w)
     q, k, v, k_len = workloads.make_inputs(w)
     import numpy as np
 
@@ -301,11 +321,163 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_bwd(args, world, w):
+    q, k, v, _ = workloads.make_inputs(w)
+    do = workloads.make_dout(w)
+    threads = os.cpu_count() or 1
+    run, flops_step, desc = bwd_oracle_sample(w, q, k, v, do, threads)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    value = flops_step * args.steps / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, world, (q.numel() + k.numel() + v.numel()) * q.element_size()),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: {desc}; {args.steps} steps"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours_bwd(args, world, rank, local, w):
+    """The backward pass (fa_bwd) of a forward computed once, untimed, by fa_fwd_ex."""
+    import ctypes
+    dev = torch.device("cuda", local)
+    q, k, v, k_len = workloads.make_inputs(w)
+    do = workloads.make_dout(w)
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    kld = None if k_len is None else k_len.to(dev)
+    o = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.float32, device=dev)
+    lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
+    fb.fa_fwd_ex(qd, kd, vd, o, lse, w.causal, w.scale, k_len=kld)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(fb.bwd_workspace_bytes(qd), 16), dtype=torch.uint8, device=dev)
+    params = fb.make_bwd_params(qd, kd, vd, o, lse, dod, dq, dk, dv, w.causal, w.scale, k_len=kld, workspace=ws)
+    lib = fb.load()
+    stream = torch.cuda.Stream(device=dev)
+    sptr = fb._stream(stream)
+    pref = ctypes.byref(params)
+
+    def launch():
+        st = lib.fa_bwd(pref, sptr)
+        if st != fb.FA_OK:
+            raise fb.FaError(st, "fa_bwd")
+
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            launch()
+    stream.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            launch()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    kernel_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
+    flops = w.flops()
+    value = flops * args.steps * world / (elapsed_ms * 1e-3) / 1e12
+
+    # end to end: inputs from pinned host memory, gradients back to it, copies timed
+    e2e = None
+    if args.e2e_steps > 0:
+        hosts = [t.pin_memory() for t in (q, k, v, do)] + [o.cpu().pin_memory(), lse.cpu().pin_memory()]
+        devs = [qd, kd, vd, dod, o, lse]
+        outs_h = [torch.empty(t.shape, dtype=torch.float32).pin_memory() for t in (dq, dk, dv)]
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for hsrc, dst in zip(hosts, devs):
+                    dst.copy_(hsrc, non_blocking=True)
+                launch()
+                for dsrc, hdst in zip((dq, dk, dv), outs_h):
+                    hdst.copy_(dsrc, non_blocking=True)
+        e2e_step()
+        stream.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        h2d = sum(t.numel() * t.element_size() for t in hosts)
+        d2h = sum(t.numel() * t.element_size() for t in outs_h)
+        e2e = {"value": flops * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "ms_per_step": e2e_ms / args.e2e_steps, "api": "fa_bwd with torch pinned-memory copies"}
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    n_elem = w.B * w.H * w.N * w.d
+    kv_elem = w.B * w.kv_heads * w.keys * w.d
+    # Q, dO, K, V (bf16) and O, lse (fp32) read; dQ, dK, dV (fp32) written once
+    alg_bytes = 2.0 * (2 * n_elem + 2 * kv_elem) + 4.0 * n_elem + 4.0 * w.B * w.H * w.N + 4.0 * (n_elem + 2 * kv_elem)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": measured_traffic(args.workload), "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "kernel": "fa_bwd_sm100_kernel + fa_bwd_prep_kernel (one event pair)", "kernel_ms": kernel_ms,
+                "algorithmic_bytes": alg_bytes, "hbm_gbs_algorithmic": alg_bytes / (kernel_ms * 1e-3) / 1e9,
+                "hbm_peak_gbs": float(peaks["hbm_gbs"])}
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        threads = os.cpu_count() or 1
+        run, f_step, desc = bwd_oracle_sample(w, q, k, v, do, threads)
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < 10.0:
+            run()
+            n += 1
+        dt = time.perf_counter() - t0
+        cpu = {"value": f_step * n / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} x {desc}, {dt:.1f} s"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, world, (q.numel() + k.numel() + v.numel() + do.numel()) * 2),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * 2,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank, local):
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (the CUDA library has no CPU path)")
     fb.load()
     w = workloads.WORKLOADS[args.workload]
+    if w.pass_ == "bwd":
+        return run_ours_bwd(args, world, rank, local, w)
     dev = torch.device("cuda", local)
     q, k, v, k_len = workloads.make_inputs(w)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)

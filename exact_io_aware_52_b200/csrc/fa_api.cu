@@ -96,6 +96,20 @@ fa_status encode_map(CUtensorMap *map, const void *base, int BH, int N, int D, i
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// 3-D map over a contiguous [B*H][N][D] fp32 tensor, box {32, 128, 1} (one
+// 128-byte column block of a 128-row tile), 128-byte swizzle: the target of
+// the backward's dQ reduce-add.
+fa_status encode_map_f32(CUtensorMap *map, void *base, int BH, int N, int D) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)N * D * 4};
+    cuuint32_t box[3] = {32, (cuuint32_t)fa::BM, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 // Validation that needs no device: shared by every entry point.
 fa_status validate(const fa_fwd_params *p) {
     if (!p) return FA_ERR_INVALID_ARGUMENT;
@@ -275,6 +289,7 @@ fa_status fa_bwd(const fa_bwd_params *p, void *stream) {
     if ((st = encode_map(&kp.tm_do, p->dout, BH, p->N, p->d)) != FA_OK) return st;
     if ((st = encode_map(&kp.tm_k, p->k, p->B * H_kv, n_k, p->d)) != FA_OK) return st;
     if ((st = encode_map(&kp.tm_v, p->v, p->B * H_kv, n_k, p->d)) != FA_OK) return st;
+    if ((st = encode_map_f32(&kp.tm_dq, p->dq, BH, p->N, p->d)) != FA_OK) return st;
     kp.lse = p->lse;
     kp.delta = static_cast<const float *>(p->workspace);
     kp.dq = p->dq;

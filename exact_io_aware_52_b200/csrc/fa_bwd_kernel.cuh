@@ -13,20 +13,26 @@
 // unit = one 128-key tile of one (b, key/value head); the unit loops over the
 // query heads that use the key/value head and over the 128-row query tiles
 // that may attend to its keys, keeping dK and dV in TMEM; each query tile's
-// dQ contribution is added to the fp32 dQ in global memory atomically.  Per
-// query tile t (products on tcgen05, bf16 operands, fp32 in TMEM):
+// dQ contribution is added to the fp32 dQ in global memory by a TMA
+// reduce-add from shared memory.  Per query tile t (products on tcgen05,
+// bf16 operands, fp32 in TMEM):
 //     S^T  = K Q_t^T      -> R_S      (keys x queries)
 //     dP^T = V dO_t^T     -> R_P
 //     P^T  = exp2(S^T sigma log2e - lse log2e)  (compute warps; bf16 over R_S)
 //     dV  += P^T dO_t     (A = P^T from TMEM, B = dO_t MN-major)
 //     dS^T = sigma P^T o (dP^T - D)  (compute warps; bf16 over R_P and, as
-//                                     the MN-major A of the next product, smem)
+//                                     the MN-major A of dQ_t, in shared memory)
 //     dK  += dS^T Q_t     (A = dS^T from TMEM, B = Q_t MN-major)
-//     dQ_t = dS K         -> R_S (A = dS MN-major from smem, B = K MN-major)
+//     dQ_t = dS K         -> R_P (A = dS MN-major, B = K MN-major)
+// Issue order: S_{t+1} right after dV_t (P_t has been read), so the scores of
+// the next tile are ready when the compute warps finish dS_t and the dQ_t
+// read-out; dP_{t+1} once dQ_t has left R_P.  dQ_t goes from TMEM through
+// the query tile's own (no longer needed) Q and dO buffers, in the 128-byte
+// swizzle of the dQ tensor map, to the reduce-add.
 // TMEM: R_S [0,128), R_P [128,256), dV [256, 256+D), dK [256+D, 256+2D).
 // Warps 0-3 compute (thread = TMEM lane: a key row of S^T, dP^T, dV, dK and a
-// query row of dQ_t), warp 4 issues the MMAs, warp 5 the TMA loads.  Every
-// wait is bounded as in the forward kernel.
+// query row of dQ_t), warp 4 issues the MMAs, warp 5 the TMA loads, warp 6 the
+// dQ reduce-adds.  Every wait is bounded as in the forward kernel.
 #pragma once
 
 #include "fa_fwd_kernel.cuh"
@@ -34,16 +40,18 @@
 namespace fa {
 namespace bwd {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kMmaWarp = 4;
 constexpr int kLoadWarp = 5;
+constexpr int kReduceWarp = 6;  // one thread issues the dQ reduce-adds
 constexpr uint32_t kColS = 0, kColP = 128, kColDV = 256;
 
 struct BwdParams {
     CUtensorMap tm_q, tm_k, tm_v, tm_do;  // Q, dO over [B*H][N][D]; K, V over [B*H_kv][Nk][D]
+    CUtensorMap tm_dq;                    // dQ fp32 over [B*H][N][D], box {32, 128, 1}, 128-byte swizzle
     const float *lse;                     // [B, H, N] from the forward
     const float *delta;                   // [B, H, N]: D_i = dO_i . O_i
-    float *dq;                            // [B, H, N, D] fp32, zeroed, accumulated atomically
+    float *dq;                            // [B, H, N, D] fp32, zeroed, accumulated by reduce-add
     float *dk, *dv;                       // [B, H_kv, Nk, D] fp32
     const int32_t *k_len;
     int32_t *status;
@@ -65,12 +73,14 @@ struct BCfg {
     static constexpr int kOffQ = kOffV + kTileBytes;      // [2]
     static constexpr int kOffDO = kOffQ + 2 * kTileBytes; // [2]
     static constexpr int kOffDS = kOffDO + 2 * kTileBytes;  // 128 keys x 128 queries bf16, MN-major A of dQ
-    static constexpr int kOffBar = kOffDS + BM * BN * 2;
+    static constexpr int kOffCol = kOffDS + BM * BN * 2;     // per-query constants of the tile: 2 x 128 fp32
+    static constexpr int kOffBar = kOffCol + 2 * BN * 4;
     static constexpr int kBarKV = 0, kBarKVEmpty = 1;
-    static constexpr int kBarSlot = 2, kBarSlotEmpty = 4;  // [2] each
-    static constexpr int kBarS = 6, kBarDP = 7, kBarPReady = 8, kBarDSReady = 9, kBarDQ = 10, kBarRSFree = 11;
-    static constexpr int kBarDKV = 12, kBarDKVFree = 13, kBarDrain = 14;
-    static constexpr int kNumBars = 15;
+    static constexpr int kBarSlot = 2, kBarSlotEmpty = 4;  // [2] each; empty: after the dQ reduce read the slot
+    static constexpr int kBarS = 6, kBarDP = 7, kBarPReady = 8, kBarDSReady = 9, kBarDQ = 10, kBarRPFree = 11;
+    static constexpr int kBarDKV = 12, kBarDKVFree = 13, kBarStage = 14, kBarColReady = 15, kBarColFree = 16;
+    static constexpr int kBarDrain = 17;
+    static constexpr int kNumBars = 18;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 4;
     // + slack to align the base to 1024 bytes; at least 117 KB so that one CTA
@@ -135,7 +145,10 @@ __device__ __forceinline__ bool compute_role(const BwdParams &p, uint64_t *bars,
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float LOG2E = 1.4426950408889634f;
     const float NEG_INF = __int_as_float(0xff800000);
+    const float POS_INF = __int_as_float(0x7f800000);
     uint8_t *s_ds = smem + C::kOffDS;
+    float *s_l2 = reinterpret_cast<float *>(smem + C::kOffCol);  // [128] lse log2(e)
+    float *s_sd = s_l2 + BN;                                      // [128] sigma D
     const uint64_t to = p.timeout_ns;
     uint32_t gt = 0;  // iterations (global): phase of the per-iteration barriers
     uint32_t gu = 0;  // units with work: phase of dkv / dkv_free
@@ -159,12 +172,25 @@ __device__ __forceinline__ bool compute_role(const BwdParams &p, uint64_t *bars,
             int bh, qt;
             iter_coord(p, u, it, bh, qt);
             const int q0 = qt * BM;
-            // lse and D of the tile's queries, read by every thread (the same
-            // addresses across a warp: one broadcast load each); queries past N
-            // count as masked
-            const float *lse_t = p.lse + (size_t)bh * p.N + q0;
-            const float *del_t = p.delta + (size_t)bh * p.N + q0;
-            const int n_valid = min(BN, p.N - q0);
+            // the tile's per-query constants into shared memory, one query per
+            // thread: lse log2(e) (+inf for queries past N or without a key, so
+            // that their P is 0) and sigma D; every thread then reads all 128
+            // with broadcast loads
+            if (gt > 0) {  // everyone has finished the previous tile's dS
+                ok = mbar_wait(&bars[C::kBarColFree], (gt - 1) & 1, abort_flag, to);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
+            {
+                const int qi = q0 + r;
+                const float l = qi < p.N ? __ldg(p.lse + (size_t)bh * p.N + qi) : NEG_INF;
+                s_l2[r] = l == NEG_INF ? POS_INF : l * LOG2E;
+                s_sd[r] = qi < p.N ? p.scale * __ldg(p.delta + (size_t)bh * p.N + qi) : 0.f;
+            }
+            mbar_arrive(&bars[C::kBarColReady]);
+            ok = mbar_wait(&bars[C::kBarColReady], gt & 1, abort_flag, to);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
             // queries [qlo, N) may attend to key kj (causal: qi >= kj - (Nk - N))
             int qlo = 0;
             if (p.causal) qlo = kj - (p.Nk - p.N);
@@ -183,15 +209,19 @@ __device__ __forceinline__ bool compute_role(const BwdParams &p, uint64_t *bars,
                 tmem_ld_wait();
                 tmem_reg_fence_f<32>(sv);
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
+                for (int c = 0; c < 32; c += 4) {
                     const int col = ch * 32 + c;
-                    const float l0 = col < n_valid ? __ldg(lse_t + col) : NEG_INF;
-                    const float l1 = col + 1 < n_valid ? __ldg(lse_t + col + 1) : NEG_INF;
-                    float p0 = ex2_approx(sv[c] * p.scale_log2 - l0 * LOG2E);
-                    float p1 = ex2_approx(sv[c + 1] * p.scale_log2 - l1 * LOG2E);
-                    if (col < c_lo || l0 == NEG_INF) p0 = 0.f;
-                    if (col + 1 < c_lo || l1 == NEG_INF) p1 = 0.f;
+                    const float4 l = *reinterpret_cast<const float4 *>(s_l2 + col);
+                    float p0 = ex2_approx(fmaf(sv[c], p.scale_log2, -l.x));
+                    float p1 = ex2_approx(fmaf(sv[c + 1], p.scale_log2, -l.y));
+                    float p2 = ex2_approx(fmaf(sv[c + 2], p.scale_log2, -l.z));
+                    float p3 = ex2_approx(fmaf(sv[c + 3], p.scale_log2, -l.w));
+                    if (col < c_lo) p0 = 0.f;
+                    if (col + 1 < c_lo) p1 = 0.f;
+                    if (col + 2 < c_lo) p2 = 0.f;
+                    if (col + 3 < c_lo) p3 = 0.f;
                     pk[col >> 1] = pack_bf16x2(p0, p1);
+                    pk[(col >> 1) + 1] = pack_bf16x2(p2, p3);
                 }
             }
             tmem_st32(tmem + lane_off + kColS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
@@ -205,62 +235,62 @@ __device__ __forceinline__ bool compute_role(const BwdParams &p, uint64_t *bars,
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            uint32_t ds[64];
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
+                uint32_t ds[16];  // dS^T for queries [32 ch, 32 ch + 32), bf16 pairs
                 float dp[32];
                 tmem_ld32f(tmem + lane_off + kColP + ch * 32, dp);
                 tmem_ld_wait();
                 tmem_reg_fence_f<32>(dp);
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
+                for (int c = 0; c < 32; c += 4) {
                     const int col = ch * 32 + c;
-                    const uint32_t pp = pk[col >> 1];
-                    const float d0 = col < n_valid ? __ldg(del_t + col) : 0.f;
-                    const float d1 = col + 1 < n_valid ? __ldg(del_t + col + 1) : 0.f;
-                    const float v0 = p.scale * bf16x2_lo(pp) * (dp[c] - d0);
-                    const float v1 = p.scale * bf16x2_hi(pp) * (dp[c + 1] - d1);
-                    ds[col >> 1] = pack_bf16x2(v0, v1);
+                    const float4 sd = *reinterpret_cast<const float4 *>(s_sd + col);
+                    const uint32_t pa = pk[col >> 1], pb = pk[(col >> 1) + 1];
+                    ds[c >> 1] = pack_bf16x2(bf16x2_lo(pa) * fmaf(dp[c], p.scale, -sd.x),
+                                             bf16x2_hi(pa) * fmaf(dp[c + 1], p.scale, -sd.y));
+                    ds[(c >> 1) + 1] = pack_bf16x2(bf16x2_lo(pb) * fmaf(dp[c + 2], p.scale, -sd.z),
+                                                   bf16x2_hi(pb) * fmaf(dp[c + 3], p.scale, -sd.w));
                 }
+                // over R_P columns [16 ch, 16 ch + 16), whose fp32 dP has been read
+                tmem_st16(tmem + lane_off + kColP + ch * 16, ds);
                 // dS as the MN-major A operand of dQ = dS K: key row r, queries
                 // [32 ch, 32 ch + 32) = 4 16-byte units of 64-query block ch / 2
                 uint8_t *blk = s_ds + (ch >> 1) * (BM * 128);
 #pragma unroll
-                for (int u4 = 0; u4 < 4; ++u4) {
-                    const int w = ch * 16 + u4 * 4;
-                    st_sw128(blk, r, (ch & 1) * 4 + u4, make_uint4(ds[w], ds[w + 1], ds[w + 2], ds[w + 3]));
-                }
+                for (int u4 = 0; u4 < 4; ++u4)
+                    st_sw128(blk, r, (ch & 1) * 4 + u4, make_uint4(ds[4 * u4], ds[4 * u4 + 1], ds[4 * u4 + 2],
+                                                                   ds[4 * u4 + 3]));
             }
-            tmem_st32(tmem + lane_off + kColP, *reinterpret_cast<uint32_t(*)[32]>(&ds[0]));
-            tmem_st32(tmem + lane_off + kColP + 32, *reinterpret_cast<uint32_t(*)[32]>(&ds[32]));
             tmem_st_wait();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // dS visible to the tensor core
             tc_fence_before();
             mbar_arrive(&bars[C::kBarDSReady]);
+            mbar_arrive(&bars[C::kBarColFree]);  // done with this tile's lse and D
 
-            // ---- dQ_t rows (TMEM lane = query q0 + r) added to dQ
+            // ---- dQ_t rows (TMEM lane = query q0 + r) into the tile's Q and dO
+            // buffers in the dQ map's swizzled layout, then reduce-added to dQ
             ok = mbar_wait(&bars[C::kBarDQ], gt & 1, abort_flag, to);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            const int qi = q0 + r;
-            float4 *dst = reinterpret_cast<float4 *>(p.dq + ((size_t)bh * p.N + qi) * D);
+            const uint32_t slot = gt & 1;
+            uint8_t *stage[2] = {smem + C::kOffQ + slot * C::kTileBytes, smem + C::kOffDO + slot * C::kTileBytes};
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_off + kColS + ch * 32, v);
+                tmem_ld32(tmem + lane_off + kColP + ch * 32, v);
                 tmem_ld_wait();
                 tmem_reg_fence(v);
-                if (qi < p.N) {
+                uint8_t *blk = stage[ch / C::kChunks] + (ch % C::kChunks) * (BM * 128);
 #pragma unroll
-                    for (int c = 0; c < 32; c += 4)
-                        atomicAdd(dst + ch * 8 + c / 4, make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                                                    __uint_as_float(v[c + 2]),
-                                                                    __uint_as_float(v[c + 3])));
-                }
+                for (int u8 = 0; u8 < 8; ++u8)
+                    st_sw128(blk, r, u8, make_uint4(v[4 * u8], v[4 * u8 + 1], v[4 * u8 + 2], v[4 * u8 + 3]));
             }
             tc_fence_before();
-            mbar_arrive(&bars[C::kBarRSFree]);
+            mbar_arrive(&bars[C::kBarRPFree]);  // R_P may take dP of the next tile
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(&bars[C::kBarStage]);  // the reduce warp adds the tile to dQ
         }
         if (!ok) break;
         // ---- dK, dV rows of the key tile
@@ -294,6 +324,39 @@ __device__ __forceinline__ bool compute_role(const BwdParams &p, uint64_t *bars,
     return ok;
 }
 
+// ------------------------------------------------------------------ dQ reduce
+// One thread: for every query tile, once the compute warps have staged dQ_t
+// in the tile's Q and dO buffers, reduce-add it to dQ through the fp32 map and
+// release the buffers to the loader after the copy engine has read them.
+template <int D>
+__device__ __forceinline__ bool reduce_role(const BwdParams &p, uint64_t *bars, volatile int *abort_flag,
+                                            uint8_t *smem) {
+    using C = BCfg<D>;
+    uint32_t gt = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+        const int t = unit_index(k);
+        if (t >= p.n_units) break;
+        const BUnit u = decode_bunit(p, t);
+        for (int it = 0; it < u.n_iter; ++it, ++gt) {
+            if (!mbar_wait(&bars[C::kBarStage], gt & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            int bh, qt;
+            iter_coord(p, u, it, bh, qt);
+            const uint32_t slot = gt & 1;
+            uint8_t *stage[2] = {smem + C::kOffQ + slot * C::kTileBytes, smem + C::kOffDO + slot * C::kTileBytes};
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch)
+                tma_reduce_add_3d(&p.tm_dq, stage[ch / C::kChunks] + (ch % C::kChunks) * (BM * 128), ch * 32,
+                                  qt * BM, bh);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+            mbar_arrive(&bars[C::kBarSlotEmpty + slot]);
+        }
+    }
+    bulk_wait_group0();  // every reduce-add has completed before the CTA exits
+    return ok;
+}
+
 // ------------------------------------------------------------------ MMA issuer
 template <int D>
 __device__ __forceinline__ bool mma_role(const BwdParams &p, uint64_t *bars, volatile int *abort_flag, uint32_t tmem,
@@ -318,46 +381,49 @@ __device__ __forceinline__ bool mma_role(const BwdParams &p, uint64_t *bars, vol
         if constexpr (D == 128) mma_ss_k128(tmem + d_col, a, b, id_sp, 0u);
         else mma_ss_k64(tmem + d_col, a, b, id_sp, 0u);
     };
+    auto wait = [&](int bar, uint32_t parity) -> bool {
+        if (!mbar_wait(&bars[bar], parity, abort_flag, to)) return false;
+        tc_fence_after();
+        return true;
+    };
     bool ok = true;
     for (int k = 0; ok; ++k) {
         const int t = unit_index(k);
         if (t >= p.n_units) break;
         const BUnit u = decode_bunit(p, t);
         if (u.n_iter == 0) continue;
-        if (!mbar_wait(&bars[C::kBarKV], gkv & 1, abort_flag, to)) { ok = false; break; }
+        if (!wait(C::kBarKV, gkv & 1)) { ok = false; break; }
         ++gkv;
-        tc_fence_after();
-        for (int it = 0; it < u.n_iter; ++it, ++gt) {
+        // scores and dP^T of the unit's first tile
+        {
             const uint32_t slot = gt & 1;
-            if (it == 0) {  // dP^T of the first tile (later ones are issued one tile ahead)
-                if (!mbar_wait(&bars[C::kBarSlot + slot], (gt >> 1) & 1, abort_flag, to)) { ok = false; break; }
-                tc_fence_after();
-                qk(kColP, v_km, do_km + slot * slot_step);
-                tc_commit(&bars[C::kBarDP]);
-            }
-            if (gt > 0 && !mbar_wait(&bars[C::kBarRSFree], (gt - 1) & 1, abort_flag, to)) { ok = false; break; }
-            tc_fence_after();
+            if (!wait(C::kBarSlot + slot, (gt >> 1) & 1)) { ok = false; break; }
             qk(kColS, k_km, q_km + slot * slot_step);
             tc_commit(&bars[C::kBarS]);
+            if (gt > 0 && !wait(C::kBarRPFree, (gt - 1) & 1)) { ok = false; break; }
+            qk(kColP, v_km, do_km + slot * slot_step);
+            tc_commit(&bars[C::kBarDP]);
+        }
+        for (int it = 0; it < u.n_iter; ++it, ++gt) {
+            const uint32_t slot = gt & 1, ns = (gt + 1) & 1;
+            const bool more = it + 1 < u.n_iter;
             // dV += P^T dO_t
-            if (!mbar_wait(&bars[C::kBarPReady], gt & 1, abort_flag, to)) { ok = false; break; }
-            if (it == 0 && gu > 0 && !mbar_wait(&bars[C::kBarDKVFree], (gu - 1) & 1, abort_flag, to)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
+            if (!wait(C::kBarPReady, gt & 1)) { ok = false; break; }
+            if (it == 0 && gu > 0 && !wait(C::kBarDKVFree, (gu - 1) & 1)) { ok = false; break; }
             mma_ts_k128(tmem + kColDV, tmem + kColS, do_mn + slot * slot_step, id_kv, it == 0 ? 0u : 1u);
-            // dK += dS^T Q_t ; dQ_t = dS K
-            if (!mbar_wait(&bars[C::kBarDSReady], gt & 1, abort_flag, to)) { ok = false; break; }
-            tc_fence_after();
+            // scores of the next tile into R_S (P_t is read by the product above, in order)
+            if (more) {
+                if (!wait(C::kBarSlot + ns, ((gt + 1) >> 1) & 1)) { ok = false; break; }
+                qk(kColS, k_km, q_km + ns * slot_step);
+                tc_commit(&bars[C::kBarS]);
+            }
+            // dK += dS^T Q_t ; dQ_t = dS K into R_P (after dK has read dS^T there)
+            if (!wait(C::kBarDSReady, gt & 1)) { ok = false; break; }
             mma_ts_k128(tmem + kColDV + D, tmem + kColP, q_mn + slot * slot_step, id_kv, it == 0 ? 0u : 1u);
-            mma_ss_mn_k128(tmem + kColS, ds_mn, k_mn, id_dq, 0u);
+            mma_ss_mn_k128(tmem + kColP, ds_mn, k_mn, id_dq, 0u);
             tc_commit(&bars[C::kBarDQ]);
-            tc_commit(&bars[C::kBarSlotEmpty + slot]);
-            if (it + 1 < u.n_iter) {  // dP^T of the next tile into R_P (dS^T there is consumed in order)
-                const uint32_t ns = (gt + 1) & 1;
-                if (!mbar_wait(&bars[C::kBarSlot + ns], ((gt + 1) >> 1) & 1, abort_flag, to)) { ok = false; break; }
-                tc_fence_after();
+            if (more) {  // dP^T of the next tile once dQ_t has been read out of R_P
+                if (!wait(C::kBarRPFree, gt & 1)) { ok = false; break; }
                 qk(kColP, v_km, do_km + ns * slot_step);
                 tc_commit(&bars[C::kBarDP]);
             } else {
@@ -380,6 +446,7 @@ __device__ __forceinline__ void load_role(const BwdParams &p, uint64_t *bars, vo
     prefetch_tensormap(&p.tm_k);
     prefetch_tensormap(&p.tm_v);
     prefetch_tensormap(&p.tm_do);
+    prefetch_tensormap(&p.tm_dq);
     const uint64_t to = p.timeout_ns;
     uint32_t gt = 0, gkv = 0;
     bool ok = true;
@@ -459,8 +526,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1) fa_bwd_sm100_kernel(const __
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
-            const bool per_row = i == C::kBarPReady || i == C::kBarDSReady || i == C::kBarRSFree ||
-                                 i == C::kBarDKVFree;
+            const bool per_row = i == C::kBarPReady || i == C::kBarDSReady || i == C::kBarRPFree ||
+                                 i == C::kBarDKVFree || i == C::kBarStage || i == C::kBarColReady ||
+                                 i == C::kBarColFree;
             mbar_init(&bars[i], per_row ? 128u : 1u);
         }
         *abort_flag = 0;
@@ -484,6 +552,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1) fa_bwd_sm100_kernel(const __
         }
     } else if (warp == bwd::kLoadWarp) {
         if (lane == 0) bwd::load_role<D>(p, bars, abort_flag, smem);
+    } else if (warp == bwd::kReduceWarp) {
+        if (lane == 0 && !bwd::reduce_role<D>(p, bars, abort_flag, smem)) bwd::record_timeout_b(p);
     }
     tc_fence_before();
     __syncthreads();

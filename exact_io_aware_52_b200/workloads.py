@@ -15,7 +15,7 @@ GPT-2 (length 1K) workloads by shape only; no dataset is involved.
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass, field
+from dataclasses import dataclass, field, replace
 
 import torch
 
@@ -35,6 +35,7 @@ class Workload:
     Nk: int | None = None              # keys (more keys than queries: cached keys); None: N
     splits: int = 0                    # key splits the benchmark uses (0: none, -1: library's choice)
     dtype: str = "bf16"                # element type of Q, K, V: "bf16" or "e4m3"
+    pass_: str = "fwd"                 # "fwd" (O and lse) or "bwd" (dQ, dK, dV for a seeded dO)
     seed: int = 0
     notes: str = field(default="", compare=False)
 
@@ -53,7 +54,11 @@ class Workload:
 
     def flops(self) -> float:
         """Nominal attention FLOPs: 4*B*H*N^2*d, halved when causal; with N_k != N,
-        4*B*H*d times the allowed (query, key) pairs (bottom-right causal mask)."""
+        4*B*H*d times the allowed (query, key) pairs (bottom-right causal mask).
+        The backward pass counts 2.5 times the forward (five products of the
+        forward's size instead of two)."""
+        if self.pass_ == "bwd":
+            return 2.5 * Workload.flops(replace(self, pass_="fwd"))
         if self.Nk is None or self.Nk == self.N:
             f = 4.0 * self.B * self.H * self.N * self.N * self.d
             return f / 2 if self.causal else f
@@ -84,7 +89,19 @@ WORKLOADS = {
     # FP8: the shape of workload 4 with E4M3 inputs (unit scales)
     9: Workload("long-context causal FP8-E4M3 B1 H32 N16384 d128", 1, 32, 16384, 128, True,
                 sample_rows_per_head=64, seed=52009, dtype="e4m3"),
+    # the backward pass of workload 4's shape, for a seeded dO ~ N(0, 1)
+    10: Workload("backward long-context causal B1 H32 N16384 d128", 1, 32, 16384, 128, True,
+                 sample_rows_per_head=64, seed=52010, pass_="bwd"),
+    # a small backward case of the same kernel (profiler captures)
+    11: Workload("backward causal B1 H8 N4096 d128", 1, 8, 4096, 128, True, seed=52011, pass_="bwd"),
 }
+
+
+def make_dout(w: Workload):
+    """The seeded upstream gradient dO ~ N(0, 1), bf16 [B, H, N, d], of a backward workload."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed + 1)
+    return torch.randn((w.B, w.H, w.N, w.d), generator=g, dtype=torch.float32).to(torch.bfloat16)
 
 
 def make_inputs(w: Workload, seed: int | None = None):

@@ -228,7 +228,7 @@ FA_EXPORT size_t fa_bwd_workspace_bytes(const fa_bwd_params *p);
 
 /*
  * fa_bwd -- two launches on `stream`: D and a zeroed dQ, then the gradients
- * (dQ accumulated in fp32 with atomic adds, one key tile per work unit).
+ * (dQ accumulated in fp32 by TMA reduce-adds, one key tile per work unit).
  * All pointers except k_len and dev_status must be 16-byte aligned.  Errors
  * as for fa_fwd_ex (d not in {64, 128}: FA_ERR_UNSUPPORTED).  dq, dk and dv
  * are deterministic up to the order of the fp32 additions into dq.

@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -22,10 +23,20 @@ constexpr int kVersion = 300;  // 0.3.0
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplits = 1024;
 
+// Scheduler words of the forward kernels' dynamic work distribution: one
+// pair per launch slot ([0] next unit, [1] CTAs done), zero at module load
+// and reset to zero by the last CTA of each launch.  A launch takes the next
+// slot round-robin, so up to kSchedSlots launches may be in flight at once
+// on one device (on any streams).
+constexpr int kSchedSlots = 64;
+static __device__ uint32_t g_sched[2 * kSchedSlots];
+std::atomic<uint32_t> g_sched_next{0};
+
 struct DeviceInfo {
     bool probed = false;
     bool supported = false;
     int num_sms = 0;
+    uint32_t *sched = nullptr;  // g_sched on this device
     bool attr_set[4][2] = {};  // [d = 64, 128, 256, 128 with E4M3 inputs][bf16 out]
     bool bwd_attr_set[2] = {};  // backward kernel, [d == 128]
 };
@@ -71,6 +82,14 @@ fa_status probe_device(int *dev_out, DeviceInfo **info_out) {
             return FA_ERR_CUDA;
         di.supported = (major == 10 && minor == 0);  // the binary is sm_100a only
         di.num_sms = sms;
+        if (di.supported) {
+            void *sp = nullptr;
+            if (cudaGetSymbolAddress(&sp, g_sched) != cudaSuccess || sp == nullptr) {
+                cudaGetLastError();
+                return FA_ERR_CUDA;
+            }
+            di.sched = static_cast<uint32_t *>(sp);
+        }
         di.probed = true;
     }
     if (!di.supported) return FA_ERR_UNSUPPORTED;
@@ -305,6 +324,17 @@ fa_status fa_bwd(const fa_bwd_params *p, void *stream) {
     kp.group = p->H / H_kv;
     kp.n_kv_tiles = (n_k + fa::BN - 1) / fa::BN;
     kp.n_units = p->B * H_kv * kp.n_kv_tiles;
+    {
+        // band of key tiles: the (key/value head, key tile) units in flight
+        // (one per SM) should span few enough heads for their Q and dO (~64 MB)
+        // to stay in L2
+        const double qdo_head = 4.0 * p->N * p->d * (double)(p->H / H_kv);
+        int heads_fit = (int)(64.0e6 / (qdo_head > 1.0 ? qdo_head : 1.0));
+        if (heads_fit < 1) heads_fit = 1;
+        int band = (di->num_sms + heads_fit - 1) / heads_fit;
+        kp.band_tiles = band < 1 ? 1 : (band > kp.n_kv_tiles ? kp.n_kv_tiles : band);
+    }
+    kp.sched = di->sched + 2 * (g_sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
     kp.causal = p->causal;
     kp.scale = p->scale;
     kp.scale_log2 = (float)((double)p->scale * 1.4426950408889634074);
@@ -362,6 +392,22 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     kp.n_splits = sp.splits;
     kp.split_tiles = sp.split_tiles;
     kp.n_units = BH * kp.n_blocks * sp.splits;
+    {
+        // band of query blocks in the unit order: the (query head, block) pairs
+        // in flight (about one per SM and split) should span few enough heads
+        // for their K and V (~64 MB) to stay in L2
+        const double kv_head = 2.0 * sp.n_k * p->d * eb / (double)(p->H / H_kv);
+        int heads_fit = (int)(64.0e6 / (kv_head > 1.0 ? kv_head : 1.0));
+        if (heads_fit < 1) heads_fit = 1;
+        const int in_flight = (di->num_sms + sp.splits - 1) / sp.splits;
+        int band = (in_flight + heads_fit - 1) / heads_fit;
+        kp.band_blocks = band < 1 ? 1 : (band > kp.n_blocks ? kp.n_blocks : band);
+        // causal units differ in cost: hand them out dynamically; equal-cost
+        // (non-causal) units keep the static snake over head-major order
+        kp.dynamic = p->causal ? 1 : 0;
+        if (!kp.dynamic) kp.band_blocks = kp.n_blocks;
+    }
+    kp.sched = di->sched + 2 * (g_sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
     kp.causal = p->causal;
     if (e4m3_in(p)) {
         // value scales: Q K^T by descale_q * descale_k (folded into the softmax

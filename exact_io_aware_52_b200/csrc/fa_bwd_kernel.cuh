@@ -58,6 +58,8 @@ struct BwdParams {
     int B, H, N, Nk, H_kv, group;
     int n_kv_tiles;                       // ceil(Nk / 128)
     int n_units;                          // B * H_kv * n_kv_tiles
+    int band_tiles;                       // key tiles per band of the unit order (see decode_bunit)
+    uint32_t *sched;                      // this launch's scheduler words: [0] next unit, [1] CTAs done
     int causal;
     float scale;                          // sigma
     float scale_log2;                     // sigma * log2(e)
@@ -80,12 +82,16 @@ struct BCfg {
     static constexpr int kBarS = 6, kBarDP = 7, kBarPReady = 8, kBarDSReady = 9, kBarDQ = 10, kBarRPFree = 11;
     static constexpr int kBarDKV = 12, kBarDKVFree = 13, kBarStage = 14, kBarColReady = 15, kBarColFree = 16;
     static constexpr int kBarDrain = 17;
-    static constexpr int kNumBars = 18;
+    static constexpr int kBarUnitFull = 18;                    // [kUnitQueue]
+    static constexpr int kBarUnitFree = 18 + kUnitQueue;       // [kUnitQueue]: compute, MMA, reduce threads
+    static constexpr int kNumBars = 18 + 2 * kUnitQueue;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 4;
+    static constexpr int kOffUnitIds = kOffAbort + 4;          // [kUnitQueue][4] ints
     // + slack to align the base to 1024 bytes; at least 117 KB so that one CTA
     // (which allocates all of TMEM) runs per SM
-    static constexpr int kSmemBytes = (kOffAbort + 4 + 1024) > 119808 ? (kOffAbort + 4 + 1024) : 119808;
+    static constexpr int kSmemBytes =
+        (kOffUnitIds + 16 * kUnitQueue + 1024) > 119808 ? (kOffUnitIds + 16 * kUnitQueue + 1024) : 119808;
     static_assert(kTileBytes % 1024 == 0, "1024-byte alignment of swizzled tiles");
     static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
     static_assert(2 * kSmemBytes > 233472, "one CTA per SM: TMEM is allocated whole");
@@ -99,10 +105,18 @@ struct BUnit {
     int n_iter;        // group * nq (0: the key tile gets no gradient)
 };
 
+// Unit numbering: the key tiles of every (b, key/value head) are cut into
+// bands of band_tiles consecutive tiles (the first tiles see the most causal
+// query tiles); units go band by band, head-major inside a band.  Units are
+// handed out dynamically in this order (the forward's unit queue).
 __device__ __forceinline__ BUnit decode_bunit(const BwdParams &p, int t) {
     BUnit u;
-    u.kvt = t % p.n_kv_tiles;
-    const int g = t / p.n_kv_tiles;
+    const int G = p.B * p.H_kv;
+    const int band = t / (p.band_tiles * G);
+    const int in_band = t - band * p.band_tiles * G;
+    const int bsz = min(p.band_tiles, p.n_kv_tiles - band * p.band_tiles);
+    const int g = in_band / bsz;
+    u.kvt = band * p.band_tiles + (in_band - g * bsz);
     u.b = g / p.H_kv;
     u.hkv = g - u.b * p.H_kv;
     u.kv0 = u.kvt * BN;
@@ -139,7 +153,8 @@ __device__ __forceinline__ void st_sw128(uint8_t *block, int r, int u, uint4 v) 
 // ------------------------------------------------------------------ compute warps
 template <int D>
 __device__ __forceinline__ bool compute_role(const BwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                             uint32_t tmem, uint8_t *smem, int warp, int lane) {
+                                             const UnitQueue &uq, uint32_t tmem, uint8_t *smem, int warp,
+                                             int lane) {
     using C = BCfg<D>;
     const int r = warp * 32 + lane;  // TMEM lane
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
@@ -154,8 +169,9 @@ __device__ __forceinline__ bool compute_role(const BwdParams &p, uint64_t *bars,
     uint32_t gu = 0;  // units with work: phase of dkv / dkv_free
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
+        const int t = unit_pop(uq, k, abort_flag, to, ok);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok || t < 0) break;
         const BUnit u = decode_bunit(p, t);
         const int kj = u.kv0 + r;  // this thread's key (rows of S^T, dP^T, dK, dV)
         const size_t kv_row = ((size_t)u.b * p.H_kv + u.hkv) * p.Nk + kj;
@@ -330,13 +346,13 @@ __device__ __forceinline__ bool compute_role(const BwdParams &p, uint64_t *bars,
 // release the buffers to the loader after the copy engine has read them.
 template <int D>
 __device__ __forceinline__ bool reduce_role(const BwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                            uint8_t *smem) {
+                                            const UnitQueue &uq, uint8_t *smem) {
     using C = BCfg<D>;
     uint32_t gt = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
+        const int t = unit_pop(uq, k, abort_flag, p.timeout_ns, ok);
+        if (!ok || t < 0) break;
         const BUnit u = decode_bunit(p, t);
         for (int it = 0; it < u.n_iter; ++it, ++gt) {
             if (!mbar_wait(&bars[C::kBarStage], gt & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
@@ -359,8 +375,8 @@ __device__ __forceinline__ bool reduce_role(const BwdParams &p, uint64_t *bars, 
 
 // ------------------------------------------------------------------ MMA issuer
 template <int D>
-__device__ __forceinline__ bool mma_role(const BwdParams &p, uint64_t *bars, volatile int *abort_flag, uint32_t tmem,
-                                         uint32_t smem_base) {
+__device__ __forceinline__ bool mma_role(const BwdParams &p, uint64_t *bars, volatile int *abort_flag,
+                                         const UnitQueue &uq, uint32_t tmem, uint32_t smem_base) {
     using C = BCfg<D>;
     const uint64_t to = p.timeout_ns;
     // K-major views (contraction over d) and MN-major views (contraction over rows)
@@ -388,8 +404,8 @@ __device__ __forceinline__ bool mma_role(const BwdParams &p, uint64_t *bars, vol
     };
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
+        const int t = unit_pop(uq, k, abort_flag, to, ok);
+        if (!ok || t < 0) break;
         const BUnit u = decode_bunit(p, t);
         if (u.n_iter == 0) continue;
         if (!wait(C::kBarKV, gkv & 1)) { ok = false; break; }
@@ -440,7 +456,7 @@ __device__ __forceinline__ bool mma_role(const BwdParams &p, uint64_t *bars, vol
 // ------------------------------------------------------------------ TMA producer
 template <int D>
 __device__ __forceinline__ void load_role(const BwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                          uint8_t *smem) {
+                                          const UnitQueue &uq, uint8_t *smem) {
     using C = BCfg<D>;
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_k);
@@ -451,8 +467,10 @@ __device__ __forceinline__ void load_role(const BwdParams &p, uint64_t *bars, vo
     uint32_t gt = 0, gkv = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
+        const int t = unit_take(uq, p.sched, p.n_units, true, k, abort_flag, to, ok);
+        if (!ok) break;
+        unit_publish(uq, k, t, 0, 0);
+        if (t < 0) break;
         const BUnit u = decode_bunit(p, t);
         if (u.n_iter == 0) continue;
         if (gkv > 0 && !mbar_wait(&bars[C::kBarKVEmpty], (gkv - 1) & 1, abort_flag, to)) { ok = false; break; }
@@ -524,12 +542,16 @@ __global__ void __launch_bounds__(bwd::kThreads, 1) fa_bwd_sm100_kernel(const __
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffAbort);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const UnitQueue uq{reinterpret_cast<volatile int *>(smem + C::kOffUnitIds), &bars[C::kBarUnitFull],
+                       &bars[C::kBarUnitFree]};
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
             const bool per_row = i == C::kBarPReady || i == C::kBarDSReady || i == C::kBarRPFree ||
                                  i == C::kBarDKVFree || i == C::kBarStage || i == C::kBarColReady ||
                                  i == C::kBarColFree;
-            mbar_init(&bars[i], per_row ? 128u : 1u);
+            // a queued unit id is read by the 128 compute threads, the MMA thread and the reduce thread
+            const bool unit_free = i >= C::kBarUnitFree && i < C::kBarUnitFree + kUnitQueue;
+            mbar_init(&bars[i], unit_free ? 130u : (per_row ? 128u : 1u));
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -543,17 +565,17 @@ __global__ void __launch_bounds__(bwd::kThreads, 1) fa_bwd_sm100_kernel(const __
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     if (warp < 4) {
-        if (!bwd::compute_role<D>(p, bars, abort_flag, tmem, smem, warp, lane)) bwd::record_timeout_b(p);
+        if (!bwd::compute_role<D>(p, bars, abort_flag, uq, tmem, smem, warp, lane)) bwd::record_timeout_b(p);
     } else if (warp == bwd::kMmaWarp) {
         if (lane == 0) {
-            if (!bwd::mma_role<D>(p, bars, abort_flag, tmem, smem_u32(smem))) bwd::record_timeout_b(p);
+            if (!bwd::mma_role<D>(p, bars, abort_flag, uq, tmem, smem_u32(smem))) bwd::record_timeout_b(p);
             tc_commit(&bars[C::kBarDrain]);
             mbar_wait_drain(&bars[C::kBarDrain], 0, p.timeout_ns);
         }
     } else if (warp == bwd::kLoadWarp) {
-        if (lane == 0) bwd::load_role<D>(p, bars, abort_flag, smem);
+        if (lane == 0) bwd::load_role<D>(p, bars, abort_flag, uq, smem);
     } else if (warp == bwd::kReduceWarp) {
-        if (lane == 0 && !bwd::reduce_role<D>(p, bars, abort_flag, smem)) bwd::record_timeout_b(p);
+        if (lane == 0 && !bwd::reduce_role<D>(p, bars, abort_flag, uq, smem)) bwd::record_timeout_b(p);
     }
     tc_fence_before();
     __syncthreads();
@@ -562,6 +584,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1) fa_bwd_sm100_kernel(const __
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if (threadIdx.x == 0) sched_release(p.sched);
 }
 
 }  // namespace fa

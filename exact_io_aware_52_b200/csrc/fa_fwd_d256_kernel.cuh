@@ -60,25 +60,26 @@ constexpr int kBarSFull = kBarEmpty + kSlots;   // [2] per score buffer
 constexpr int kBarPFull = kBarSFull + 2;        // [2] per score buffer (128 arrivals)
 constexpr int kBarODone = kBarPFull + 2;        // [2] per parity of the P V product index
 constexpr int kBarOFree = kBarODone + 2;        // 128 arrivals
-constexpr int kBarDrain = kBarOFree + 1;
+constexpr int kBarUnitFull = kBarOFree + 1;               // [kUnitQueue]
+constexpr int kBarUnitFree = kBarUnitFull + kUnitQueue;    // [kUnitQueue], 128 softmax threads + MMA thread
+constexpr int kBarDrain = kBarUnitFree + kUnitQueue;
 constexpr int kNumBars = kBarDrain + 1;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemSlot + 4;
-constexpr int kSmemUsed = kOffAbort + 4;
+constexpr int kOffUnitIds = kOffAbort + 4;
+constexpr int kSmemUsed = kOffUnitIds + 16 * kUnitQueue;
 constexpr int kSmemBytes = kSmemUsed + 1024;  // + slack to align the base to 1024 bytes
 static_assert(kHalfBytes % 1024 == 0 && kBlockBytes % 1024 == 0, "1024-byte alignment of swizzled tiles");
 static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
 static_assert(2 * kSmemBytes > 233472, "one CTA per SM: TMEM is allocated whole");
 
 // Unit t -> (b, h, query tile, split) and the key tiles [lo, lo + n) that some
-// row of the tile may attend to: as decode_unit with one query tile per unit
-// (p.n_blocks = ceil(N / 128)).
+// row of the tile may attend to: as decode_unit (same banded order) with one
+// query tile per unit (p.n_blocks = ceil(N / 128)).
 __device__ __forceinline__ UnitCoord decode_unit1(const FwdParams &p, int t) {
     UnitCoord u;
     u.split = t % p.n_splits;
-    const int r = t / p.n_splits;
-    u.blk = p.n_blocks - 1 - r % p.n_blocks;
-    u.bh = r / p.n_blocks;
+    band_decode(p, t / p.n_splits, u.bh, u.blk);
     u.b = u.bh / p.H;
     u.bh_kv = u.b * p.H_kv + (u.bh - u.b * p.H) / p.group;
     u.lo = u.split * p.split_tiles;
@@ -109,7 +110,7 @@ __device__ __forceinline__ bool wait_pv_upto(uint64_t *bars, uint32_t &waited, l
 // ------------------------------------------------------------------ softmax
 template <bool O_BF16>
 __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                             uint32_t tmem, int warp, int lane) {
+                                             const UnitQueue &uq, uint32_t tmem, int warp, int lane) {
     const int row_in_tile = warp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float LN2 = 0.69314718055994530942f;
@@ -121,8 +122,9 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
     uint32_t tl = 0;      // units with work (o_free phase)
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
+        const int t = p.dynamic ? unit_pop(uq, k, abort_flag, to, ok) : unit_static(p, k);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok || t < 0) break;
         const UnitCoord u = decode_unit1(p, t);
         const int row = u.blk * kUnitRows + row_in_tile;
         const bool row_valid = row < p.N;
@@ -235,7 +237,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
 
 // ------------------------------------------------------------------ MMA issuer
 __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                         uint32_t tmem, uint32_t q_addr, uint32_t ring_addr) {
+                                         const UnitQueue &uq, uint32_t tmem, uint32_t q_addr, uint32_t ring_addr) {
     const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
     const uint32_t idesc_pv = idesc_bf16_f32(BM, 128, true);
     const uint64_t q_desc = sw128_desc(q_addr, 16, 1024);
@@ -286,10 +288,10 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
 
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
-        const UnitCoord u = decode_unit1(p, t);
-        const int n = u.n[0];
+        int n = 0;  // dynamic: the key-tile count comes with the id (the TMA warp decoded the unit)
+        const int t = p.dynamic ? unit_pop(uq, k, abort_flag, to, ok, &n) : unit_static(p, k);
+        if (!ok || t < 0) break;
+        if (!p.dynamic) n = decode_unit1(p, t).n[0];
         if (n == 0) continue;
         if (!mbar_wait(&bars[kBarQFull], tq & 1, abort_flag, to)) { ok = false; break; }
         ++tq;
@@ -313,7 +315,7 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
 
 // ------------------------------------------------------------------ TMA producer
 __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                          uint8_t *sQ, uint8_t *ring) {
+                                          const UnitQueue &uq, uint8_t *sQ, uint8_t *ring) {
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_k);
     prefetch_tensormap(&p.tm_v);
@@ -336,9 +338,14 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
         return true;
     };
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
+        const int t = p.dynamic ? unit_take(p, uq, k, abort_flag, to, ok) : unit_static(p, k);
+        if (!ok) break;
+        if (t < 0) {
+            if (p.dynamic) unit_publish(uq, k, -1, 0, 0);
+            break;
+        }
         const UnitCoord u = decode_unit1(p, t);
+        if (p.dynamic) unit_publish(uq, k, t, u.n[0], 0);
         const int n = u.n[0];
         if (n == 0) continue;
         if (tq > 0 && !mbar_wait(&bars[kBarQEmpty], (tq - 1) & 1, abort_flag, to)) {
@@ -384,10 +391,12 @@ __global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_d256_kernel(const __
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    const UnitQueue uq{reinterpret_cast<volatile int *>(smem + kOffUnitIds), &bars[kBarUnitFull], &bars[kBarUnitFree]};
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) {
             const bool per_row = (i >= kBarPFull && i < kBarPFull + 2) || i == kBarOFree;
-            mbar_init(&bars[i], per_row ? 128u : 1u);
+            const bool unit_free = i >= kBarUnitFree && i < kBarUnitFree + kUnitQueue;
+            mbar_init(&bars[i], unit_free ? 129u : (per_row ? 128u : 1u));
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -402,15 +411,15 @@ __global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_d256_kernel(const __
     const uint32_t tmem = *tmem_slot;
 
     if (warp < d256::kSoftmaxWarps) {
-        if (!d256::softmax_role<O_BF16>(p, bars, abort_flag, tmem, warp, lane)) record_timeout(p);
+        if (!d256::softmax_role<O_BF16>(p, bars, abort_flag, uq, tmem, warp, lane)) record_timeout(p);
     } else if (warp == d256::kMmaWarp) {
         if (lane == 0) {
-            if (!d256::mma_role(p, bars, abort_flag, tmem, smem_u32(sQ), smem_u32(ring))) record_timeout(p);
+            if (!d256::mma_role(p, bars, abort_flag, uq, tmem, smem_u32(sQ), smem_u32(ring))) record_timeout(p);
             tc_commit(&bars[kBarDrain]);
             mbar_wait_drain(&bars[kBarDrain], 0, p.timeout_ns);
         }
     } else if (warp == d256::kLoadWarp) {
-        if (lane == 0) d256::load_role(p, bars, abort_flag, sQ, ring);
+        if (lane == 0) d256::load_role(p, bars, abort_flag, uq, sQ, ring);
     }
 
     tc_fence_before();
@@ -420,6 +429,7 @@ __global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_d256_kernel(const __
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if (threadIdx.x == 0 && p.dynamic) sched_release(p.sched);
 }
 
 }  // namespace fa

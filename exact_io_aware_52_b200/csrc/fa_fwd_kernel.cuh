@@ -59,13 +59,14 @@ constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;   // warps 10-11 only complete the third warpgroup
 constexpr int kThreads = 384;
 // Register split (setmaxnreg): the launch gives 384 x 168; the two softmax
-// warpgroups take 216 each and the MMA/TMA warpgroup keeps 72:
-// 256 * 216 + 128 * 72 = 64512 = 384 * 168, and 216 + 216 + 72 <= 512 per lane
+// warpgroups take 224 each and the MMA/TMA warpgroup keeps 56:
+// 256 * 224 + 128 * 56 = 64512 = 384 * 168, and 224 + 224 + 56 <= 512 per lane
 // on every SM sub-partition (one warp of each warpgroup per sub-partition).
-constexpr int kSoftmaxRegs = 216;
-constexpr int kControlRegs = 72;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kControlRegs = 56;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
+constexpr int kUnitQueue = 4;  // depth of the shared-memory queue of work-unit ids
 constexpr int kStatusTimeout = 5;  // FA_ERR_DEVICE_TIMEOUT
 // Of every kPolyPeriod key pairs of a score row, the last kPolyPairs take
 // their exponentials from the FMA-pipe polynomial, the rest from MUFU ex2.
@@ -105,6 +106,9 @@ struct FwdParams {
     int n_splits;                  // key-range splits per query block (1: none)
     int split_tiles;               // key tiles per split
     int n_units;                   // B * H * n_blocks * n_splits
+    int band_blocks;               // query blocks per band of the unit order (see decode_unit)
+    int dynamic;                   // units handed out by the counter (1) or in the static snake order (0)
+    uint32_t *sched;               // this launch's scheduler words: [0] next unit, [1] CTAs done
     int causal;
     float scale_log2;              // scale * log2(e)
     float tau;                     // rescale threshold in log2 units (<= 0: rescale on any growth)
@@ -140,11 +144,14 @@ struct Cfg {
     static constexpr int kBarOFinal = kBarPFull + 2;         // [2]
     static constexpr int kBarOFree = kBarOFinal + 2;         // [2]
     static constexpr int kBarPHalf = kBarOFree + 2;          // [2] P of keys [0, 64) in TMEM
-    static constexpr int kBarDrain = kBarPHalf + 2;
+    static constexpr int kBarUnitFull = kBarPHalf + 2;       // [kUnitQueue]
+    static constexpr int kBarUnitFree = kBarUnitFull + kUnitQueue;  // [kUnitQueue]
+    static constexpr int kBarDrain = kBarUnitFree + kUnitQueue;
     static constexpr int kNumBars = kBarDrain + 1;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 4;
-    static constexpr int kSmemUsed = kOffAbort + 4;
+    static constexpr int kOffUnitIds = kOffAbort + 4;                // [kUnitQueue][4] ints
+    static constexpr int kSmemUsed = kOffUnitIds + 16 * kUnitQueue;
     static constexpr int kSmemBytes = kSmemUsed + 1024;  // + slack to align the base to 1024 bytes
     static_assert(kChunkBytes % 1024 == 0 && kTileBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
@@ -159,24 +166,111 @@ struct UnitCoord {
     int nmax;
 };
 
-// Work unit k of this CTA: bands of gridDim.x consecutive units, walked in
-// alternating direction so that per-CTA work evens out when the units'
-// costs fall band by band (causal masking puts the longest units first).
+// Static schedule (the backward kernel): work unit k of this CTA is taken from
+// bands of gridDim.x consecutive units, walked in alternating direction.
 __device__ __forceinline__ int unit_index(int k) {
     const int G = gridDim.x, c = blockIdx.x;
     return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-// Units are numbered head-major (the CTAs working at one time share a few
-// heads' K and V in L2), longest (causal) query blocks first within a head,
-// key splits innermost.  Query tile x of the unit covers the key tiles of the
-// unit's split that some row of the tile may attend to.
+// ------------------------------------------------------------------ work distribution
+// Units are handed out dynamically, in index order, from a per-launch counter
+// in global memory: whichever CTA is free takes the next one, so the causal
+// units' unequal costs even out at the end of the launch.  Inside a CTA the
+// TMA warp (which runs ahead) takes the ids and passes them to the other
+// roles through a small shared-memory queue.
+struct UnitQueue {
+    volatile int *ids;  // [kUnitQueue][4]: unit id, then two words the producer may attach
+    uint64_t *full;     // [kUnitQueue], one arrival: the producer has written the entry
+    uint64_t *free;     // [kUnitQueue], one arrival per consuming thread
+};
+
+// Producer (one thread), step 1: the id of this CTA's k-th unit, or -1 when
+// none is left (ok turns false when the wait for a free entry times out).
+__device__ __forceinline__ int unit_take(const UnitQueue &q, uint32_t *counter, int n_units, bool dynamic, int k,
+                                         volatile int *abort_flag, uint64_t timeout_ns, bool &ok) {
+    const int slot = k % kUnitQueue;
+    if (k >= kUnitQueue && !mbar_wait(&q.free[slot], ((k / kUnitQueue) - 1) & 1, abort_flag, timeout_ns)) {
+        ok = false;
+        return -1;
+    }
+    // dynamic: the first unit of CTA c is unit c (no wait at the start), the
+    // rest come from the counter after the gridDim.x units taken that way;
+    // static: the snake order of unit_index
+    const int t = !dynamic ? unit_index(k)
+                           : (k == 0 ? (int)blockIdx.x : (int)gridDim.x + (int)atomicAdd(counter, 1u));
+    return t < n_units ? t : -1;
+}
+
+// Producer, step 2: publish entry k (id t, -1 included so that consumers stop,
+// and two attached words).
+__device__ __forceinline__ int unit_take(const FwdParams &p, const UnitQueue &q, int k, volatile int *abort_flag,
+                                         uint64_t timeout_ns, bool &ok) {
+    return unit_take(q, p.sched, p.n_units, p.dynamic != 0, k, abort_flag, timeout_ns, ok);
+}
+
+// Static order: every role computes its k-th unit itself (no queue).
+__device__ __forceinline__ int unit_static(const FwdParams &p, int k) {
+    const int t = unit_index(k);
+    return t < p.n_units ? t : -1;
+}
+
+__device__ __forceinline__ void unit_publish(const UnitQueue &q, int k, int t, int a, int b) {
+    volatile int *e = q.ids + 4 * (k % kUnitQueue);
+    e[0] = t;
+    e[1] = a;
+    e[2] = b;
+    mbar_arrive(&q.full[k % kUnitQueue]);  // release: the entry is visible to whoever acquires the phase
+}
+
+// Consumer: entry k (returns the id, -1: no more units; a and b the attached
+// words); ok turns false if the wait times out or the CTA is aborting.
+__device__ __forceinline__ int unit_pop(const UnitQueue &q, int k, volatile int *abort_flag, uint64_t timeout_ns,
+                                        bool &ok, int *a = nullptr, int *b = nullptr) {
+    const int slot = k % kUnitQueue;
+    if (!mbar_wait(&q.full[slot], (k / kUnitQueue) & 1, abort_flag, timeout_ns)) {
+        ok = false;
+        return -1;
+    }
+    volatile int *e = q.ids + 4 * slot;
+    const int t = e[0];
+    if (a) *a = e[1];
+    if (b) *b = e[2];
+    mbar_arrive(&q.free[slot]);
+    return t;
+}
+
+// The last CTA to finish resets the launch's scheduler words for the next
+// launch that uses them (every CTA has taken its last id by then).
+__device__ __forceinline__ void sched_release(uint32_t *sched) {
+    __threadfence();
+    if (atomicAdd(sched + 1, 1u) == gridDim.x - 1) {
+        atomicExch(sched, 0u);
+        atomicExch(sched + 1, 0u);
+    }
+}
+
+// Unit numbering: the query blocks of every (b, h) are cut into bands of
+// band_blocks consecutive blocks, longest (causal) first; units go band by
+// band, head-major inside a band, longest block first within a head, key
+// splits innermost.  A band of one block is block-major order (the best
+// balance), a band of all blocks head-major order (the CTAs at work share few
+// heads' K and V in L2); the host picks the band so that the heads in flight
+// fit in L2.  Query tile x of the unit covers the key tiles of the unit's
+// split that some row of the tile may attend to.
+__device__ __forceinline__ void band_decode(const FwdParams &p, int r, int &bh, int &blk) {
+    const int BH = p.B * p.H;
+    const int band = r / (p.band_blocks * BH);
+    const int in_band = r - band * p.band_blocks * BH;
+    const int bsz = min(p.band_blocks, p.n_blocks - band * p.band_blocks);
+    bh = in_band / bsz;
+    blk = p.n_blocks - 1 - (band * p.band_blocks + (in_band - bh * bsz));
+}
+
 __device__ __forceinline__ UnitCoord decode_unit(const FwdParams &p, int t) {
     UnitCoord u;
     u.split = t % p.n_splits;
-    const int r = t / p.n_splits;
-    u.blk = p.n_blocks - 1 - r % p.n_blocks;
-    u.bh = r / p.n_blocks;
+    band_decode(p, t / p.n_splits, u.bh, u.blk);
     u.b = u.bh / p.H;
     u.bh_kv = u.b * p.H_kv + (u.bh - u.b * p.H) / p.group;
     u.lo = u.split * p.split_tiles;
@@ -327,7 +421,7 @@ constexpr float kF8Shift = 8.f;
 
 template <int D, bool O_BF16, bool F8>
 __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                             uint32_t tmem, int x, int warp, int lane) {
+                                             const UnitQueue &uq, uint32_t tmem, int x, int warp, int lane) {
     using C = Cfg<D, F8>;
     const int row_in_tile = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -344,8 +438,9 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
     uint32_t tl = 0;  // units in which this query tile had work (o_final / o_free phase)
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
+        const int t = p.dynamic ? unit_pop(uq, k, abort_flag, p.timeout_ns, ok) : unit_static(p, k);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok || t < 0) break;
         const UnitCoord u = decode_unit(p, t);
         const int row = u.blk * kUnitRows + x * BM + row_in_tile;
         const bool row_valid = row < p.N;
@@ -473,7 +568,8 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
 // ------------------------------------------------------------------ MMA issuer
 template <int D, bool F8>
 __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                         uint32_t tmem, uint32_t q_addr, uint32_t k_addr, uint32_t v_addr) {
+                                         const UnitQueue &uq, uint32_t tmem, uint32_t q_addr, uint32_t k_addr,
+                                         uint32_t v_addr) {
     using C = Cfg<D, F8>;
     const uint32_t idesc_qk = F8 ? idesc_e4m3_f32(BM, BN, false) : idesc_bf16_f32(BM, BN, false);
     const uint32_t idesc_pv = F8 ? idesc_e4m3_f32(BM, D, true) : idesc_bf16_f32(BM, D, true);
@@ -530,9 +626,11 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
 
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
-        const UnitCoord u = decode_unit(p, t);
+        UnitCoord u;  // dynamic: the key-tile counts come with the id (the TMA warp decoded the unit)
+        const int t = p.dynamic ? unit_pop(uq, k, abort_flag, to, ok, &u.n[0], &u.n[1]) : unit_static(p, k);
+        if (!ok || t < 0) break;
+        if (!p.dynamic) u = decode_unit(p, t);
+        u.nmax = max(u.n[0], u.n[1]);
         if (u.nmax == 0) continue;
         if (!mbar_wait(&bars[C::kBarQFull], tq & 1, abort_flag, to)) { ok = false; break; }
         ++tq;
@@ -573,7 +671,7 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
 // ------------------------------------------------------------------ TMA producer
 template <int D, bool F8>
 __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                          uint8_t *sQ, uint8_t *sK, uint8_t *sV) {
+                                          const UnitQueue &uq, uint8_t *sQ, uint8_t *sK, uint8_t *sV) {
     using C = Cfg<D, F8>;
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_k);
@@ -582,9 +680,14 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
     uint32_t tq = 0, gk = 0, gv = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        const int t = unit_index(k);
-        if (t >= p.n_units) break;
+        const int t = p.dynamic ? unit_take(p, uq, k, abort_flag, to, ok) : unit_static(p, k);
+        if (!ok) break;
+        if (t < 0) {
+            if (p.dynamic) unit_publish(uq, k, -1, 0, 0);
+            break;
+        }
         const UnitCoord u = decode_unit(p, t);
+        if (p.dynamic) unit_publish(uq, k, t, u.n[0], u.n[1]);
         if (u.nmax == 0) continue;
         if (tq > 0 && !mbar_wait(&bars[C::kBarQEmpty], (tq - 1) & 1, abort_flag, to)) {
             ok = false;
@@ -658,12 +761,16 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    const UnitQueue uq{reinterpret_cast<volatile int *>(smem + C::kOffUnitIds), &bars[C::kBarUnitFull],
+                       &bars[C::kBarUnitFree]};
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
             const bool per_row = (i >= C::kBarPFull && i < C::kBarPFull + 2) ||
                                  (i >= C::kBarOFree && i < C::kBarOFree + 2) ||
                                  (i >= C::kBarPHalf && i < C::kBarPHalf + 2);
-            mbar_init(&bars[i], per_row ? 128u : 1u);
+            // a queued unit id is read by the 256 softmax threads and the MMA thread
+            const bool unit_free = i >= C::kBarUnitFree && i < C::kBarUnitFree + kUnitQueue;
+            mbar_init(&bars[i], unit_free ? 2u * 128u + 1u : (per_row ? 128u : 1u));
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -679,20 +786,20 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
 
     if (warp < kSoftmaxWarps) {
         setmaxnreg_inc<kSoftmaxRegs>();
-        if (!softmax_role<D, O_BF16, F8>(p, bars, abort_flag, tmem, warp >> 2, warp, lane)) record_timeout(p);
+        if (!softmax_role<D, O_BF16, F8>(p, bars, abort_flag, uq, tmem, warp >> 2, warp, lane)) record_timeout(p);
     } else {
         setmaxnreg_dec<kControlRegs>();
     }
     if (warp == kMmaWarp) {
         if (lane == 0) {
-            if (!mma_role<D, F8>(p, bars, abort_flag, tmem, smem_u32(sQ), smem_u32(sK), smem_u32(sV)))
+            if (!mma_role<D, F8>(p, bars, abort_flag, uq, tmem, smem_u32(sQ), smem_u32(sK), smem_u32(sV)))
                 record_timeout(p);
             // drain: no MMA may still be running when TMEM is released
             tc_commit(&bars[C::kBarDrain]);
             mbar_wait_drain(&bars[C::kBarDrain], 0, p.timeout_ns);
         }
     } else if (warp == kLoadWarp) {
-        if (lane == 0) load_role<D, F8>(p, bars, abort_flag, sQ, sK, sV);
+        if (lane == 0) load_role<D, F8>(p, bars, abort_flag, uq, sQ, sK, sV);
     }
 
     tc_fence_before();
@@ -702,6 +809,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if (threadIdx.x == 0 && p.dynamic) sched_release(p.sched);
 }
 
 }  // namespace fa

@@ -155,7 +155,10 @@ FA_EXPORT int fa_fwd_suggest_splits(const fa_fwd_params *p);
 
 /*
  * fa_fwd_ex -- the forward pass with key padding, output dtype and a status
- * word.  On a device-side timeout the kernel stores FA_ERR_DEVICE_TIMEOUT in
+ * word.  Causal problems hand their work units out through a per-launch
+ * counter held by the library (64 slots per device, taken round-robin): at
+ * most 64 causal fa_fwd / fa_fwd_ex / fa_bwd launches may be in flight on one
+ * device at the same time, on any streams.  On a device-side timeout the kernel stores FA_ERR_DEVICE_TIMEOUT in
  * *dev_status, stops, writes NaN to the rows of the tile it was working on
  * and leaves the rows of unprocessed tiles unwritten.
  */

@@ -237,3 +237,41 @@ def test_status_word_stays_clear():
     lse = torch.empty(1, 2, 256, device=dev)
     fb.fa_fwd_ex(q.to(dev), k.to(dev), v.to(dev), o, lse, False, 0.125, dev_status=st, timeout_ms=500)
     assert fb.read_device_status(st) == fb.FA_OK
+
+
+# ------------------------------------------------------------ dynamic work distribution
+def test_scheduler_slots_are_reused_cleanly():
+    """150 causal launches in a row cycle through the library's 64 scheduler
+    slots twice: every launch must see its slot reset (bit-identical outputs)."""
+    q, k, v = rand_inputs(2, 6, 1000, 128, seed=18)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o_ref, l_ref = fb.attention(qd, kd, vd, True, 0.088)
+    o = torch.empty_like(o_ref)
+    lse = torch.empty_like(l_ref)
+    for i in range(150):
+        o.fill_(float("nan"))
+        fb.fa_fwd_ex(qd, kd, vd, o, lse, True, 0.088)
+        if i % 37 == 0 or i == 149:
+            assert torch.equal(o, o_ref) and torch.equal(lse, l_ref), i
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref)
+
+
+def test_concurrent_streams():
+    """Causal launches on four streams at once take different scheduler slots
+    and all give the single-stream result."""
+    q, k, v = rand_inputs(1, 8, 2048, 128, seed=19)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o_ref, l_ref = fb.attention(qd, kd, vd, True, 0.088)
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    outs = [(torch.full_like(o_ref, float("nan")), torch.full_like(l_ref, float("nan"))) for _ in streams]
+    torch.cuda.synchronize()
+    for _ in range(5):
+        for s, (o, lse) in zip(streams, outs):
+            with torch.cuda.stream(s):
+                fb.fa_fwd_ex(qd, kd, vd, o, lse, True, 0.088, stream=s)
+    torch.cuda.synchronize()
+    for o, lse in outs:
+        assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)

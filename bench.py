@@ -29,6 +29,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -129,7 +130,11 @@ class ClockSampler:
 
     def __init__(self, device_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        # raw samples go to FA_BENCH_OUT (default: the system temp dir); the
+        # JSON line carries their summary
+        out_dir = os.environ.get("FA_BENCH_OUT") or tempfile.gettempdir()
+        os.makedirs(out_dir, exist_ok=True)
+        self.path = os.path.join(out_dir, f"clocks_rank{device_index}.csv")
         props = torch.cuda.get_device_properties(device_index)
         self.bus = None  # "BB:DD" (bus:device, hex) of the GPU this rank uses
         try:

@@ -592,7 +592,7 @@ def run_ours(args, world, rank, local):
                 "frac": achieved / peak, "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
                 "traffic": traffic,
                 "peak_source": f"{peak_src} {peak_label}" + (" x 2 (nominal FP8/BF16 dense ratio)" if fp8 else ""),
-                "kernel": ("fa_fwd_d256_kernel" if w.d == 256 else "fa_fwd_sm100_kernel")
+                "kernel": ("fa_fwd_onetile_kernel" if w.d == 256 else "fa_fwd_sm100_kernel")
                           + (" + fa_combine_kernel (split pass and merge, one event pair)" if splits > 1 else ""),
                 "kernel_ms": kernel_ms,
                 "algorithmic_bytes": alg_bytes, "hbm_gbs_algorithmic": alg_bytes / (kernel_ms * 1e-3) / 1e9,

@@ -54,7 +54,8 @@ bool e4m3_in(const fa_fwd_params *p) { return p->in_dtype == FA_IN_E4M3; }
 bool valid_descale(float x) { return std::isfinite(x) && x >= 0.f; }
 float descale(float x) { return x > 0.f ? x : 1.f; }
 
-// Query rows per work unit: two 128-row tiles for d <= 128, one for d = 256.
+// Query rows per work unit: two 128-row tiles for d <= 128 (the ping-pong
+// kernel), one for d = 256 (the one-tile kernel).
 int unit_rows(int d) { return d == 256 ? fa::d256::kUnitRows : fa::kUnitRows; }
 
 fa_status load_encoder() {
@@ -192,8 +193,8 @@ template <int D, bool BF16, bool F8 = false>
 fa_status launch(const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t stream) {
     constexpr bool kD256 = D == 256;
     constexpr int kD = kD256 ? 128 : D;
-    auto kern = kD256 ? fa::fa_fwd_d256_kernel<BF16> : fa::fa_fwd_sm100_kernel<kD, BF16, F8>;
-    const int smem = kD256 ? fa::d256::kSmemBytes : fa::Cfg<kD, F8>::kSmemBytes;
+    auto kern = kD256 ? fa::fa_fwd_onetile_kernel<256, BF16> : fa::fa_fwd_sm100_kernel<kD, BF16, F8>;
+    const int smem = kD256 ? fa::d256::Cfg1<256>::kSmemBytes : fa::Cfg<kD, F8>::kSmemBytes;
     const int threads = kD256 ? fa::d256::kThreads : fa::kThreads;
     {
         std::lock_guard<std::mutex> lk(g_mu);

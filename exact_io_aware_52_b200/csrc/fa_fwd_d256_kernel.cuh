@@ -31,6 +31,12 @@
 //
 // Warps: 0-3 softmax (thread t owns row t of the tile), 4 MMA issuer (one
 // thread), 5 TMA producer (one thread).  192 threads, up to 255 registers each.
+//
+// The layout is written for any d that is a multiple of 128 up to 256 (Cfg1<D>:
+// D / 128 half tiles per operand, a ring as deep as shared memory allows).
+// Only d = 256 is instantiated: at d = 128 this design (six ring slots, one
+// query tile) measured about 11% slower on a B200 than the two-query-tile
+// ping-pong kernel of fa_fwd_kernel.cuh, with bit-identical outputs.
 #pragma once
 
 #include "fa_fwd_kernel.cuh"
@@ -38,40 +44,47 @@
 namespace fa {
 namespace d256 {
 
-constexpr int D = 256;
 constexpr int kUnitRows = BM;                 // one query tile per work unit
 constexpr int kHalfBytes = BM * 128 * 2;      // a 128 x 128 bf16 half tile
 constexpr int kBlockBytes = BM * 128;         // one 64-column (128-byte) block of it
-constexpr int kSlots = 5;                     // operand ring depth in half tiles
 constexpr int kSoftmaxWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kLoadWarp = 5;
 constexpr int kThreads = 192;
 constexpr uint32_t kColO = 256;
 
-constexpr int kOffQ = 0;                              // Q_lo, Q_hi
-constexpr int kOffRing = kOffQ + 2 * kHalfBytes;      // kSlots half tiles
-constexpr int kOffBar = kOffRing + kSlots * kHalfBytes;
-constexpr int kBarQFull = 0;
-constexpr int kBarQEmpty = 1;
-constexpr int kBarFull = 2;                     // [kSlots]
-constexpr int kBarEmpty = kBarFull + kSlots;    // [kSlots]
-constexpr int kBarSFull = kBarEmpty + kSlots;   // [2] per score buffer
-constexpr int kBarPFull = kBarSFull + 2;        // [2] per score buffer (128 arrivals)
-constexpr int kBarODone = kBarPFull + 2;        // [2] per parity of the P V product index
-constexpr int kBarOFree = kBarODone + 2;        // 128 arrivals
-constexpr int kBarUnitFull = kBarOFree + 1;               // [kUnitQueue]
-constexpr int kBarUnitFree = kBarUnitFull + kUnitQueue;    // [kUnitQueue], 128 softmax threads + MMA thread
-constexpr int kBarDrain = kBarUnitFree + kUnitQueue;
-constexpr int kNumBars = kBarDrain + 1;
-constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr int kOffAbort = kOffTmemSlot + 4;
-constexpr int kOffUnitIds = kOffAbort + 4;
-constexpr int kSmemUsed = kOffUnitIds + 16 * kUnitQueue;
-constexpr int kSmemBytes = kSmemUsed + 1024;  // + slack to align the base to 1024 bytes
-static_assert(kHalfBytes % 1024 == 0 && kBlockBytes % 1024 == 0, "1024-byte alignment of swizzled tiles");
-static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
-static_assert(2 * kSmemBytes > 233472, "one CTA per SM: TMEM is allocated whole");
+// Layout for head dimension D (128 or 256): Q is D / 128 half tiles, every
+// K_j and V_j D / 128 half tiles through the ring, whose depth is what the
+// rest of shared memory holds.
+template <int D>
+struct Cfg1 {
+    static_assert(D == 128 || D == 256, "one-tile kernel: d = 128 or 256");
+    static constexpr int kHalves = D / 128;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffRing = kOffQ + kHalves * kHalfBytes;
+    static constexpr int kSlots = (232448 - 1024 - 512 - kOffRing) / kHalfBytes;  // 5 for d = 256, 6 for 128
+    static constexpr int kOffBar = kOffRing + kSlots * kHalfBytes;
+    static constexpr int kBarQFull = 0;
+    static constexpr int kBarQEmpty = 1;
+    static constexpr int kBarFull = 2;                     // [kSlots]
+    static constexpr int kBarEmpty = kBarFull + kSlots;    // [kSlots]
+    static constexpr int kBarSFull = kBarEmpty + kSlots;   // [2] per score buffer
+    static constexpr int kBarPFull = kBarSFull + 2;        // [2] per score buffer (128 arrivals)
+    static constexpr int kBarODone = kBarPFull + 2;        // [2] per parity of the P V product index
+    static constexpr int kBarOFree = kBarODone + 2;        // 128 arrivals
+    static constexpr int kBarUnitFull = kBarOFree + 1;               // [kUnitQueue]
+    static constexpr int kBarUnitFree = kBarUnitFull + kUnitQueue;   // [kUnitQueue], softmax threads + MMA thread
+    static constexpr int kBarDrain = kBarUnitFree + kUnitQueue;
+    static constexpr int kNumBars = kBarDrain + 1;
+    static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+    static constexpr int kOffAbort = kOffTmemSlot + 4;
+    static constexpr int kOffUnitIds = kOffAbort + 4;
+    static constexpr int kSmemUsed = kOffUnitIds + 16 * kUnitQueue;
+    static constexpr int kSmemBytes = kSmemUsed + 1024;  // + slack to align the base to 1024 bytes
+    static_assert(kHalfBytes % 1024 == 0 && kBlockBytes % 1024 == 0, "1024-byte alignment of swizzled tiles");
+    static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
+    static_assert(2 * kSmemBytes > 233472, "one CTA per SM: TMEM is allocated whole");
+};
 
 // Unit t -> (b, h, query tile, split) and the key tiles [lo, lo + n) that some
 // row of the tile may attend to: as decode_unit (same banded order) with one
@@ -98,19 +111,22 @@ __device__ __forceinline__ UnitCoord decode_unit1(const FwdParams &p, int t) {
 // `upto` (global count over the CTA's units) not yet waited for.  Product i
 // completes phase i / 2 of o_done[i % 2]; at most one phase per barrier is
 // ever outstanding (see the issue order above), so the parity is exact.
+template <int D>
 __device__ __forceinline__ bool wait_pv_upto(uint64_t *bars, uint32_t &waited, long long upto,
                                              volatile int *abort_flag, uint64_t to) {
+    using C = Cfg1<D>;
     while ((long long)waited <= upto) {
-        if (!mbar_wait(&bars[kBarODone + (waited & 1)], (waited >> 1) & 1, abort_flag, to)) return false;
+        if (!mbar_wait(&bars[C::kBarODone + (waited & 1)], (waited >> 1) & 1, abort_flag, to)) return false;
         ++waited;
     }
     return true;
 }
 
 // ------------------------------------------------------------------ softmax
-template <bool O_BF16>
+template <int D, bool O_BF16>
 __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
                                              const UnitQueue &uq, uint32_t tmem, int warp, int lane) {
+    using C = Cfg1<D>;
     const int row_in_tile = warp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float LN2 = 0.69314718055994530942f;
@@ -144,7 +160,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         for (int j = 0; j < n; ++j, ++gs) {
             const uint32_t buf = gs & 1;
             const uint32_t t_s = tmem + lane_off + buf * 128u;
-            ok = mbar_wait(&bars[kBarSFull + buf], (gs >> 1) & 1, abort_flag, to);
+            ok = mbar_wait(&bars[C::kBarSFull + buf], (gs >> 1) & 1, abort_flag, to);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
@@ -182,7 +198,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             // the products before this tile's predecessor are complete (the
             // commit behind S ready covers them): consume their phases
             const bool any_resc = __any_sync(0xffffffffu, resc);
-            ok = wait_pv_upto(bars, waited, (long long)gs - (any_resc ? 1 : 2), abort_flag, to);
+            ok = wait_pv_upto<D>(bars, waited, (long long)gs - (any_resc ? 1 : 2), abort_flag, to);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             if (any_resc) {
@@ -206,10 +222,10 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             lr += lrs;
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&bars[kBarPFull + buf]);
+            mbar_arrive(&bars[C::kBarPFull + buf]);
         }
         if (ok) {
-            ok = wait_pv_upto(bars, waited, (long long)gs - 1, abort_flag, to);
+            ok = wait_pv_upto<D>(bars, waited, (long long)gs - 1, abort_flag, to);
             ok = __all_sync(0xffffffffu, ok);
         }
         if (!ok) {
@@ -229,15 +245,17 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         }
         if (row_valid) p.lse[row_id] = empty ? NEG_INF : (m_ref + log2f(l)) * LN2;
         tc_fence_before();
-        mbar_arrive(&bars[kBarOFree]);
+        mbar_arrive(&bars[C::kBarOFree]);
         ++tl;
     }
     return ok;
 }
 
 // ------------------------------------------------------------------ MMA issuer
+template <int D>
 __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
                                          const UnitQueue &uq, uint32_t tmem, uint32_t q_addr, uint32_t ring_addr) {
+    using C = Cfg1<D>;
     const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
     const uint32_t idesc_pv = idesc_bf16_f32(BM, 128, true);
     const uint64_t q_desc = sw128_desc(q_addr, 16, 1024);
@@ -251,37 +269,47 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
     uint32_t tl = 0;   // units with work (o_free phase)
 
     auto take = [&](uint32_t &slot) -> bool {
-        slot = g % kSlots;
-        const bool r = mbar_wait(&bars[kBarFull + slot], (g / kSlots) & 1, abort_flag, to);
+        slot = g % C::kSlots;
+        const bool r = mbar_wait(&bars[C::kBarFull + slot], (g / C::kSlots) & 1, abort_flag, to);
         ++g;
         return r;
     };
+    // S_b = sum over the halves h of Q_h K_h^T (K_j's halves in consecutive ring slots)
     auto qk = [&]() -> bool {
-        uint32_t s0, s1;
-        if (!take(s0) || !take(s1)) return false;
+        uint32_t sl[C::kHalves];
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h)
+            if (!take(sl[h])) return false;
         tc_fence_after();
         const uint32_t d = tmem + (gs & 1) * 128u;
-        mma_ss_k128(d, q_desc, k_desc + ((s0 * kHalfBytes) >> 4), idesc_qk, 0u);
-        mma_ss_k128(d, q_desc + (kHalfBytes >> 4), k_desc + ((s1 * kHalfBytes) >> 4), idesc_qk, 1u);
-        tc_commit(&bars[kBarSFull + (gs & 1)]);
-        tc_commit(&bars[kBarEmpty + s0]);
-        tc_commit(&bars[kBarEmpty + s1]);
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h)
+            mma_ss_k128(d, q_desc + ((h * kHalfBytes) >> 4), k_desc + ((sl[h] * kHalfBytes) >> 4), idesc_qk,
+                        h > 0 ? 1u : 0u);
+        tc_commit(&bars[C::kBarSFull + (gs & 1)]);
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h) tc_commit(&bars[C::kBarEmpty + sl[h]]);
         ++gs;
         return true;
     };
     auto pv = [&](bool first) -> bool {
         const uint32_t buf = gpv & 1;
-        if (!mbar_wait(&bars[kBarPFull + buf], (gpv >> 1) & 1, abort_flag, to)) return false;
-        if (first && tl > 0 && !mbar_wait(&bars[kBarOFree], (tl - 1) & 1, abort_flag, to)) return false;
-        uint32_t s0, s1;
-        if (!take(s0) || !take(s1)) return false;
+        if (!mbar_wait(&bars[C::kBarPFull + buf], (gpv >> 1) & 1, abort_flag, to)) return false;
+        if (first && tl > 0 && !mbar_wait(&bars[C::kBarOFree], (tl - 1) & 1, abort_flag, to)) return false;
+        uint32_t sl[C::kHalves];
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h)
+            if (!take(sl[h])) return false;
         tc_fence_after();
         const uint32_t a = tmem + buf * 128u;
-        mma_ts_k128(tmem + kColO, a, v_desc + ((s0 * kHalfBytes) >> 4), idesc_pv, first ? 0u : 1u);
-        mma_ts_k128(tmem + kColO + 128u, a, v_desc + ((s1 * kHalfBytes) >> 4), idesc_pv, first ? 0u : 1u);
-        tc_commit(&bars[kBarODone + buf]);
-        tc_commit(&bars[kBarEmpty + s0]);
-        tc_commit(&bars[kBarEmpty + s1]);
+        // O_h (+)= P V_h: columns [128 h, 128 h + 128) of O
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h)
+            mma_ts_k128(tmem + kColO + 128u * h, a, v_desc + ((sl[h] * kHalfBytes) >> 4), idesc_pv,
+                        first ? 0u : 1u);
+        tc_commit(&bars[C::kBarODone + buf]);
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h) tc_commit(&bars[C::kBarEmpty + sl[h]]);
         ++gpv;
         return true;
     };
@@ -293,13 +321,13 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
         if (!ok || t < 0) break;
         if (!p.dynamic) n = decode_unit1(p, t).n[0];
         if (n == 0) continue;
-        if (!mbar_wait(&bars[kBarQFull], tq & 1, abort_flag, to)) { ok = false; break; }
+        if (!mbar_wait(&bars[C::kBarQFull], tq & 1, abort_flag, to)) { ok = false; break; }
         ++tq;
         tc_fence_after();
         int jq = 0;  // score tiles of this unit issued
         auto qk_next = [&]() -> bool {
             if (!qk()) return false;
-            if (++jq == n) tc_commit(&bars[kBarQEmpty]);  // Q no longer read in this unit
+            if (++jq == n) tc_commit(&bars[C::kBarQEmpty]);  // Q no longer read in this unit
             return true;
         };
         if (!qk_next()) { ok = false; break; }
@@ -314,24 +342,26 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
 }
 
 // ------------------------------------------------------------------ TMA producer
+template <int D>
 __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
                                           const UnitQueue &uq, uint8_t *sQ, uint8_t *ring) {
+    using C = Cfg1<D>;
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_k);
     prefetch_tensormap(&p.tm_v);
     const uint64_t to = p.timeout_ns;
     uint32_t tq = 0, g = 0;
     bool ok = true;
-    // key tile `kt` of K or V as two half tiles (d columns [0,128) and [128,256))
+    // key tile `kt` of K or V as D / 128 half tiles (d columns [128 h, 128 h + 128))
     auto load_tile = [&](const CUtensorMap *map, int kt, int bh_kv) -> bool {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint32_t slot = g % kSlots, round = g / kSlots;
-            if (round > 0 && !mbar_wait(&bars[kBarEmpty + slot], (round - 1) & 1, abort_flag, to)) return false;
-            mbar_arrive_expect_tx(&bars[kBarFull + slot], kHalfBytes);
+        for (int h = 0; h < C::kHalves; ++h) {
+            const uint32_t slot = g % C::kSlots, round = g / C::kSlots;
+            if (round > 0 && !mbar_wait(&bars[C::kBarEmpty + slot], (round - 1) & 1, abort_flag, to)) return false;
+            mbar_arrive_expect_tx(&bars[C::kBarFull + slot], kHalfBytes);
 #pragma unroll
             for (int c = 0; c < 2; ++c)
-                tma_load_3d(ring + slot * kHalfBytes + c * kBlockBytes, map, &bars[kBarFull + slot], h * 128 + c * 64,
+                tma_load_3d(ring + slot * kHalfBytes + c * kBlockBytes, map, &bars[C::kBarFull + slot], h * 128 + c * 64,
                             kt * BN, bh_kv);
             ++g;
         }
@@ -348,14 +378,14 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
         if (p.dynamic) unit_publish(uq, k, t, u.n[0], 0);
         const int n = u.n[0];
         if (n == 0) continue;
-        if (tq > 0 && !mbar_wait(&bars[kBarQEmpty], (tq - 1) & 1, abort_flag, to)) {
+        if (tq > 0 && !mbar_wait(&bars[C::kBarQEmpty], (tq - 1) & 1, abort_flag, to)) {
             ok = false;
             break;
         }
-        mbar_arrive_expect_tx(&bars[kBarQFull], 2 * kHalfBytes);
+        mbar_arrive_expect_tx(&bars[C::kBarQFull], C::kHalves * kHalfBytes);
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-            tma_load_3d(sQ + c * kBlockBytes, &p.tm_q, &bars[kBarQFull], c * 64, u.blk * kUnitRows, u.bh);
+        for (int c = 0; c < 2 * C::kHalves; ++c)
+            tma_load_3d(sQ + c * kBlockBytes, &p.tm_q, &bars[C::kBarQFull], c * 64, u.blk * kUnitRows, u.bh);
         ++tq;
         // the order the MMA issuer takes them: K_0, K_1, V_0, K_2, V_1, ..., V_{n-1}
         if (!load_tile(&p.tm_k, u.lo, u.bh_kv)) { ok = false; break; }
@@ -367,35 +397,36 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
     }
     if (!ok) record_timeout(p);
     // drain: every copy this thread issued has landed before the CTA may exit
-    if (tq > 0) mbar_wait_drain(&bars[kBarQFull], (tq - 1) & 1, to);
-    const uint32_t nr = g < (uint32_t)kSlots ? g : (uint32_t)kSlots;
+    if (tq > 0) mbar_wait_drain(&bars[C::kBarQFull], (tq - 1) & 1, to);
+    const uint32_t nr = g < (uint32_t)C::kSlots ? g : (uint32_t)C::kSlots;
     for (uint32_t i = 0; i < nr; ++i) {
         const uint32_t gi = g - 1 - i;
-        mbar_wait_drain(&bars[kBarFull + gi % kSlots], (gi / kSlots) & 1, to);
+        mbar_wait_drain(&bars[C::kBarFull + gi % C::kSlots], (gi / C::kSlots) & 1, to);
     }
 }
 
 }  // namespace d256
 
-template <bool O_BF16>
-__global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_d256_kernel(const __grid_constant__ FwdParams p) {
+template <int D, bool O_BF16>
+__global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_onetile_kernel(const __grid_constant__ FwdParams p) {
     using namespace d256;
+    using C = Cfg1<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t *sQ = smem + kOffQ;
-    uint8_t *ring = smem + kOffRing;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmemSlot);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
+    uint8_t *sQ = smem + C::kOffQ;
+    uint8_t *ring = smem + C::kOffRing;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffAbort);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    const UnitQueue uq{reinterpret_cast<volatile int *>(smem + kOffUnitIds), &bars[kBarUnitFull], &bars[kBarUnitFree]};
+    const UnitQueue uq{reinterpret_cast<volatile int *>(smem + C::kOffUnitIds), &bars[C::kBarUnitFull], &bars[C::kBarUnitFree]};
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNumBars; ++i) {
-            const bool per_row = (i >= kBarPFull && i < kBarPFull + 2) || i == kBarOFree;
-            const bool unit_free = i >= kBarUnitFree && i < kBarUnitFree + kUnitQueue;
+        for (int i = 0; i < C::kNumBars; ++i) {
+            const bool per_row = (i >= C::kBarPFull && i < C::kBarPFull + 2) || i == C::kBarOFree;
+            const bool unit_free = i >= C::kBarUnitFree && i < C::kBarUnitFree + kUnitQueue;
             mbar_init(&bars[i], unit_free ? 129u : (per_row ? 128u : 1u));
         }
         *abort_flag = 0;
@@ -411,15 +442,15 @@ __global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_d256_kernel(const __
     const uint32_t tmem = *tmem_slot;
 
     if (warp < d256::kSoftmaxWarps) {
-        if (!d256::softmax_role<O_BF16>(p, bars, abort_flag, uq, tmem, warp, lane)) record_timeout(p);
+        if (!d256::softmax_role<D, O_BF16>(p, bars, abort_flag, uq, tmem, warp, lane)) record_timeout(p);
     } else if (warp == d256::kMmaWarp) {
         if (lane == 0) {
-            if (!d256::mma_role(p, bars, abort_flag, uq, tmem, smem_u32(sQ), smem_u32(ring))) record_timeout(p);
-            tc_commit(&bars[kBarDrain]);
-            mbar_wait_drain(&bars[kBarDrain], 0, p.timeout_ns);
+            if (!d256::mma_role<D>(p, bars, abort_flag, uq, tmem, smem_u32(sQ), smem_u32(ring))) record_timeout(p);
+            tc_commit(&bars[C::kBarDrain]);
+            mbar_wait_drain(&bars[C::kBarDrain], 0, p.timeout_ns);
         }
     } else if (warp == d256::kLoadWarp) {
-        if (lane == 0) d256::load_role(p, bars, abort_flag, uq, sQ, ring);
+        if (lane == 0) d256::load_role<D>(p, bars, abort_flag, uq, sQ, ring);
     }
 
     tc_fence_before();

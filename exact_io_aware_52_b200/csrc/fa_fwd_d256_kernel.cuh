@@ -214,15 +214,27 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
                     tmem_st32(t_o + ch * 32, r);
                 }
             }
-            exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
-            tmem_st32(t_s + 0, pk0);
-            exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
-            tmem_st32(t_s + 32, pk1);
-            l += ls.x + ls.y;
-            lr += lrs;
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars[C::kBarPFull + buf]);
+            if constexpr (kLateSums) {
+                exp_half_p<0>(s, p.scale_log2, -m_ref, pk0, ls);
+                tmem_st32(t_s + 0, pk0);
+                exp_half_p<1>(s, p.scale_log2, -m_ref, pk1, ls);
+                tmem_st32(t_s + 32, pk1);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bars[C::kBarPFull + buf]);
+                l += ls.x + ls.y;
+                lr += rounded_sum(pk0, pk1);
+            } else {
+                exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
+                tmem_st32(t_s + 0, pk0);
+                exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
+                tmem_st32(t_s + 32, pk1);
+                l += ls.x + ls.y;
+                lr += lrs;
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bars[C::kBarPFull + buf]);
+            }
         }
         if (ok) {
             ok = wait_pv_upto<D>(bars, waited, (long long)gs - 1, abort_flag, to);

@@ -78,6 +78,12 @@ constexpr int kPolyPairs = 0;
 // P to bf16: round to nearest even (cvt) when false; truncation (keep the
 // high half of each fp32 word, one byte permute per pair) when true.
 constexpr bool kPackTruncate = false;
+// The tile's sum of the bf16-rounded probabilities (two mixed-precision adds
+// per pair) is taken after "P ready", from the packed pairs, instead of
+// between the exponentials, so that the tensor core gets P sooner; the
+// unrounded sum (one packed add per pair) stays beside the exponentials.
+constexpr bool kLateSums = true;
+static_assert(!kLateSums || (kPolyPairs == 0 && !kPackTruncate), "late sums: MUFU exponentials, rounded P");
 // P V in two halves of 64 keys: the softmax releases P for keys [0, 64) as
 // soon as it is in TMEM, so the tensor core multiplies that half while the
 // softmax computes the other, and only P V for keys [64, 128) plus the next
@@ -400,6 +406,35 @@ __device__ __forceinline__ void exp_half(const float *s, float scale_log2, float
     lrs = ((b[0] + b[1]) + (b[2] + b[3])) + (bb.x + bb.y);
 }
 
+// Probabilities of keys [64H, 64H+64) as in exp_half, without the rounded
+// sum: pk holds the bf16 pairs, `ls` gains the unrounded values.
+template <int H>
+__device__ __forceinline__ void exp_half_p(const float *s, float scale_log2, float neg_m, uint32_t (&pk)[32],
+                                           float2 &ls) {
+    const float2 sl2 = make_float2(scale_log2, scale_log2);
+    const float2 nm = make_float2(neg_m, neg_m);
+    float2 a[4] = {ls, make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+        const float2 xx = __ffma2_rn(make_float2(s[64 * H + c], s[64 * H + c + 1]), sl2, nm);
+        const float2 pp = make_float2(ex2_approx(xx.x), ex2_approx(xx.y));
+        a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], pp);
+        pk[c >> 1] = pack_bf16x2(pp.x, pp.y);
+    }
+    ls = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+}
+
+// Sum of a tile's 128 bf16 probabilities (two per word of pk0 and pk1).
+__device__ __forceinline__ float rounded_sum(const uint32_t (&pk0)[32], const uint32_t (&pk1)[32]) {
+    float b[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        b[i & 3] = add_bf16x2_to(b[i & 3], pk0[i]);
+        b[(i + 2) & 3] = add_bf16x2_to(b[(i + 2) & 3], pk1[i]);
+    }
+    return (b[0] + b[1]) + (b[2] + b[3]);
+}
+
 // E4M3 probabilities of one 128-key score row: p = 2^(s * scale_log2 - m)
 // summed unrounded into `ls` and rounded to E4M3, four keys per 32-bit
 // column (key 4c + i in byte i of column c).
@@ -533,6 +568,16 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             if constexpr (F8) {
                 exp_e4m3(s, p.scale_log2, kF8Shift - m_ref, pk0, ls);
                 tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
+            } else if constexpr (kLateSums) {
+                exp_half_p<0>(s, p.scale_log2, -m_ref, pk0, ls);
+                tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
+                if constexpr (kSplitPV<D>) {
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(p_half);
+                }
+                exp_half_p<1>(s, p.scale_log2, -m_ref, pk1, ls);
+                tmem_st32(t_s + 32, pk1);
             } else {
                 exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
                 tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
@@ -544,11 +589,19 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
                 exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
                 tmem_st32(t_s + 32, pk1);
             }
-            l += ls.x + ls.y;
-            lr += lrs;
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(p_full);
+            if constexpr (!F8 && kLateSums) {
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(p_full);
+                l += ls.x + ls.y;
+                lr += rounded_sum(pk0, pk1);
+            } else {
+                l += ls.x + ls.y;
+                lr += lrs;
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(p_full);
+            }
         }
         if (ok) {
             ok = mbar_wait(o_final, tl & 1, abort_flag, p.timeout_ns);

@@ -1,7 +1,7 @@
 """Pins for the fp64 backward oracle (attn_bwd_oracle.c): checks against facts
 that do not come from the backward oracle itself.  Each pin takes a backward
 library handle so that the same checks run against deliberately broken builds
-(``test_oracle_bwd_mutants.py``).
+(``test_bwd_pins_catch_mutant`` in ``test_oracle_bwd.py``).
 
 Sources of truth:
 * a library routine: torch's float64 autograd through scaled_dot_product_attention

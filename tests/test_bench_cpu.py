@@ -1,0 +1,128 @@
+"""Host-side arithmetic of the benchmark's JSON line, checked on the CPU against
+closed forms and brute-force counts: the nominal FLOP counts, the algorithmic
+HBM bytes of one launch, the choice of the tensor peak, and the rule that a
+committed DRAM-traffic record is reported only for the device sources it was
+taken on."""
+import os
+
+import numpy as np
+import pytest
+
+import bench
+from exact_io_aware_52_b200 import workloads
+
+
+def _allowed_pairs(N, Nk, causal, k_len=None):
+    """Brute force: (query, key) pairs the mask allows (bottom-right causal alignment)."""
+    i = np.arange(N)[:, None]
+    j = np.arange(Nk)[None, :]
+    m = np.ones((N, Nk), dtype=bool)
+    if causal:
+        m &= j <= i + (Nk - N)
+    if k_len is not None:
+        m &= j < k_len
+    return int(m.sum())
+
+
+def test_flops_square_is_the_nominal_count():
+    w = workloads.custom(2, 3, 300, 64, causal=False)
+    assert w.flops() == 4.0 * 2 * 3 * 300 * 300 * 64
+    wc = workloads.custom(2, 3, 300, 64, causal=True)
+    assert wc.flops() == w.flops() / 2
+
+
+@pytest.mark.parametrize("N,Nk,causal", [(100, 900, True), (256, 131072, True), (37, 50, False), (5, 3, True)])
+def test_flops_rectangular_counts_allowed_pairs(N, Nk, causal):
+    w = workloads.custom(1, 2, N, 128, causal=causal, Nk=Nk)
+    assert w.flops() == 4.0 * 1 * 2 * 128 * _allowed_pairs(N, Nk, causal)
+
+
+def test_backward_flops_are_two_and_a_half_forward():
+    f = workloads.WORKLOADS[4]
+    b = workloads.WORKLOADS[10]
+    assert (b.B, b.H, b.N, b.d, b.causal) == (f.B, f.H, f.N, f.d, f.causal)
+    assert b.flops() == 2.5 * f.flops()
+
+
+def test_algorithmic_bytes_long_context():
+    w = workloads.WORKLOADS[4]  # B1 H32 N16384 d128, bf16 in, fp32 O
+    n = 1 * 32 * 16384 * 128
+    expect = 2 * n + 2 * 2 * n + 4 * n + 4 * 32 * 16384
+    assert bench.algorithmic_bytes(w, None) == expect
+
+
+def test_algorithmic_bytes_key_padding_and_groups():
+    w = workloads.custom(3, 8, 200, 64, causal=False, H_kv=2, Nk=500)
+    k_len = [500, 0, 777]  # clamped to [0, N_k]
+    n = 3 * 8 * 200 * 64
+    kv_rows = 2 * (500 + 0 + 500)
+    expect = 2 * n + 2 * 2 * kv_rows * 64 + 4 * n + 4 * 3 * 8 * 200
+    assert bench.algorithmic_bytes(w, k_len) == expect
+
+
+def test_algorithmic_bytes_e4m3_inputs_are_one_byte():
+    w = workloads.WORKLOADS[9]
+    n = w.B * w.H * w.N * w.d
+    assert bench.algorithmic_bytes(w, None) == n + 2 * n + 4 * n + 4 * w.B * w.H * w.N
+
+
+def test_tensor_peak_sustained_only_for_long_regions():
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    peak, label, burst, sustained = bench.tensor_peak(peaks, 999.9)
+    assert (peak, burst, sustained) == (1600.0, 1600.0, 1400.0) and "burst" in label
+    peak, label, _, _ = bench.tensor_peak(peaks, 1000.0)
+    assert peak == 1400.0 and "sustained" in label
+    peak, _, burst, sustained = bench.tensor_peak(peaks, 5000.0, ratio=2.0)
+    assert (peak, burst, sustained) == (2800.0, 3200.0, 2800.0)
+    # without a sustained figure the burst one stands in
+    assert bench.tensor_peak({"bf16_tflops": 1500.0}, 2000.0)[0] == 1500.0
+
+
+def _fake_tree(root, body=b"kernel v1"):
+    csrc = os.path.join(root, "exact_io_aware_52_b200", "csrc")
+    os.makedirs(csrc, exist_ok=True)
+    os.makedirs(os.path.join(root, "profiles"), exist_ok=True)
+    for name in ("a.cuh", "b.cuh"):
+        with open(os.path.join(csrc, name), "wb") as f:
+            f.write(body + name.encode())
+
+
+def _record(root, workload, source_hash, total):
+    with open(os.path.join(root, "profiles", "k_traffic.txt"), "w") as f:
+        f.write("# a comment line\n")
+        f.write("sources a.cuh b.cuh\n")
+        f.write(f"source_hash {source_hash}\nworkload {workload}\n")
+        f.write(f"dram_bytes_read 1\ndram_bytes_write 2\ndram_bytes_per_launch {total}\n")
+
+
+def test_traffic_record_follows_the_device_sources(tmp_path, monkeypatch):
+    root = str(tmp_path)
+    _fake_tree(root)
+    monkeypatch.setattr(bench, "ROOT", root)
+    h = bench.kernel_source_hash(["a.cuh", "b.cuh"])
+    _record(root, 4, h, 123456)
+    assert bench.measured_traffic(4) == 123456.0
+    assert bench.measured_traffic(8) is None  # another workload
+    _fake_tree(root, body=b"kernel v2")  # the kernel changed since the capture
+    assert bench.measured_traffic(4) is None
+    _record(root, 4, "0000000000000000", 5)
+    assert bench.measured_traffic(4) is None
+
+
+def test_committed_records_name_existing_sources():
+    """Every committed traffic record lists device sources that exist and a
+    16-hex-digit hash (whether it matches is decided at run time)."""
+    import glob
+    paths = glob.glob(os.path.join(bench.ROOT, "profiles", "*traffic.txt"))
+    assert paths
+    for path in paths:
+        rec = {}
+        for line in open(path):
+            if line.startswith("#") or not line.strip():
+                continue
+            k, _, v = line.partition(" ")
+            rec[k] = v.strip()
+        for name in rec["sources"].split():
+            assert os.path.isfile(os.path.join(bench.ROOT, "exact_io_aware_52_b200", "csrc", name)), (path, name)
+        assert len(rec["source_hash"]) == 16 and int(rec["source_hash"], 16) >= 0
+        assert float(rec["dram_bytes_per_launch"]) == float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])

@@ -1,7 +1,7 @@
 // fa_bwd_kernel.cuh -- gradients of exact attention on sm_100a.
 //
 // The pages report the method's training speed-ups (page "FlashAttention
-// (ES)", section "Impacto en el rendimiento") without a backward algorithm;
+// (ES)", section "Resultados empiricos") without a backward algorithm;
 // this is the derivative of the forward definition ("El problema de la
 // atencion estandar") computed IO-aware the way the forward is: tiles in
 // shared memory and TMEM, P recomputed from Q, K and the forward's lse rather

@@ -25,7 +25,7 @@
  *   o       : fp32  [B, H, N, d]  (fa_fwd; fa_fwd_ex may select bf16)
  *   lse     : fp32  [B, H, N]
  *   k_len   : int32 [B]  (fa_fwd_ex only; key j of batch b is masked iff
- *             j >= k_len[b]; values are clamped to [0, N] on the device)
+ *             j >= k_len[b]; values are clamped to [0, N_k] on the device)
  * Mask: causal masks key j for query i when j > i + N_k - N (j > i when
  * N_k = N).  A row with no allowed key gets O = 0, lse = -inf.
  *
@@ -197,7 +197,7 @@ FA_EXPORT int fa_version(void);
 /*
  * Backward pass: the gradients of the forward's O with respect to q, k and v
  * for a given dO.  The pages report training speed-ups of the method (page
- * "FlashAttention (ES)", section "Impacto en el rendimiento") but give no
+ * "FlashAttention (ES)", section "Resultados empiricos") but give no
  * backward algorithm; this is the derivative of the definition of section
  * "El problema de la atencion estandar", with P recomputed from q, k and the
  * forward's lse:

@@ -6,7 +6,7 @@
  * (the CUDA library) never links, loads or calls it, and the two share no code.
  *
  * The pages report training speed-ups of the method (page "FlashAttention
- * (ES)", section "Impacto en el rendimiento") but give no backward algorithm,
+ * (ES)", section "Resultados empiricos") but give no backward algorithm,
  * so what is computed here is the plain derivative of the forward definition
  * of section "El problema de la atencion estandar".  With
  *     S = sigma Q K^T (+ mask),  P = softmax_rows(S),  O = P V

@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` are the only callers.  The CUDA product path
 never imports this package, and this package imports nothing from it.
 
-Two pieces, both written from the page "FlashAttention (ES)":
+Three pieces, all written from the page "FlashAttention (ES)":
 
 * ``attention_f64`` -- the plain definition of attention (section "El problema
   de la atencion estandar", the Attention equation, with the masking step of

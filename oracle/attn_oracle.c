@@ -55,7 +55,7 @@ static double bf16_bits_to_double(uint16_t bits) {
  *   q       : bf16 bit patterns, contiguous [B, H, N, d]   (N queries)
  *   k, v    : bf16 bit patterns, contiguous [B, H_kv, Nk, d] (Nk keys); H_kv divides H
  *   k_len   : NULL, or int32[B]; key j of batch b is masked iff j >= k_len[b]
- *             (values outside [0, N] are clamped to it)
+ *             (values outside [0, Nk] are clamped to it)
  *   causal  : nonzero masks key j for query i when j > i + Nk - N
  *   scale   : the float multiplier applied to q.k (1/sqrt(d_k) in the
  *             definition); widened to double

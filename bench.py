@@ -44,6 +44,14 @@ DEFAULT_WORKLOAD = 4  # long-context causal B1 H32 N16384 d128: the tensor-bound
 METRIC = "attention fwd TFLOP/s (bf16, 1xB200) and % of dense BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["fa_fwd_kernel.cuh", "sm100_ptx.cuh"]  # device code of the d <= 128 kernel (default record)
+# Dense bf16 tensor FLOPs per SM per clock of tcgen05 kind::f16 (one 128x128x128
+# product group every 512 cycles); times the SM count and the sampled SM clock it
+# gives the clock-derived dense peak, the second denominator of every fraction.
+SM_TENSOR_FLOP_PER_CLK = 8192
+# The other workloads of the spec table, measured in the same invocation
+# as the headline (one `per_config` entry each).
+PER_CONFIG = (1, 2, 3, 5)
+PER_CONFIG_MIN_MS = 300.0  # each per-config timed region lasts at least this long (clock samples)
 
 
 def parse():
@@ -55,6 +63,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
     return ap.parse_args()
 
 
@@ -78,6 +87,43 @@ def tensor_peak(peaks: dict, elapsed_ms: float, ratio: float = 1.0):
     if elapsed_ms >= 1000.0:
         return sustained, "bf16_tflops_sustained (timed region >= 1 s back to back)", burst, sustained
     return burst, "bf16_tflops (burst; timed region < 1 s)", burst, sustained
+
+
+def clock_peak_tflops(num_sms: int, sm_mhz: float, ratio: float = 1.0) -> float:
+    """Dense tensor peak at a given SM clock: SMs x 8192 FLOP/clk x clock (x the
+    nominal dense ratio of another operand type)."""
+    return num_sms * SM_TENSOR_FLOP_PER_CLK * sm_mhz * 1e6 * ratio / 1e12
+
+
+def percentiles(xs) -> dict:
+    """Median, p10, p90 (linear interpolation between order statistics) and mean."""
+    v = sorted(float(x) for x in xs)
+    if not v:
+        return {"median": None, "p10": None, "p90": None, "mean": None, "n": 0}
+
+    def q(f):
+        pos = f * (len(v) - 1)
+        lo = int(math.floor(pos))
+        hi = min(lo + 1, len(v) - 1)
+        return v[lo] + (v[hi] - v[lo]) * (pos - lo)
+    return {"median": q(0.5), "p10": q(0.1), "p90": q(0.9), "mean": sum(v) / len(v), "n": len(v)}
+
+
+def effective_flops(w, k_len) -> float:
+    """4*d FLOPs per (query, key) pair the mask allows, keys beyond each batch
+    element's length excluded (the work the kernel cannot skip; equals
+    w.flops() without key padding, up to the causal diagonal)."""
+    if k_len is None:
+        return w.flops()
+    N, Nk = w.N, w.keys
+    tot = 0
+    for b in range(w.B):
+        L = max(0, min(Nk, int(k_len[b])))
+        if w.causal:
+            tot += sum(max(0, min(L, i + 1 + Nk - N)) for i in range(N))
+        else:
+            tot += N * L
+    return 4.0 * w.H * w.d * tot
 
 
 def kernel_source_hash(sources=None) -> str:
@@ -490,6 +536,111 @@ def run_ours_bwd(args, world, rank, local, w):
     print(json.dumps(line), flush=True)
 
 
+def time_graph_launches(launch, stream, dev, min_launches: int, min_ms: float, est_us: float):
+    """Device time per launch of `launch` from CUDA-graph replays: a graph of G
+    back-to-back launches (G chosen so one replay lasts about half a
+    millisecond or more), replayed R times, each replay bracketed by CUDA
+    events on the launching stream.  The graph removes the host's per-call
+    cost, which is larger than the kernel on the small workloads.  Returns
+    (per-launch ms of each replay, G, R, total ms)."""
+    group = int(min(100, max(1, math.ceil(500.0 / max(est_us, 1.0)))))
+    reps = max(math.ceil(min_launches / group), math.ceil(min_ms * 1e3 / (max(est_us, 1.0) * group)), 5)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(group):
+            launch()
+    g.replay()
+    stream.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for a, b in ev:
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        t1.record(stream)
+    stream.synchronize()
+    per = [a.elapsed_time(b) / group for a, b in ev]
+    total = t0.elapsed_time(t1)
+    del g
+    return per, group, reps, total
+
+
+def measure_per_config(args, local, peaks, num_sms):
+    """The other spec workloads, each measured on this device right after
+    the headline: device time per launch (median, p10, p90 over graph
+    replays), TFLOP/s at the median, and the fraction of the measured peak
+    (burst or sustained by the region's length) and of the clock-derived
+    peak at the region's median SM clock."""
+    dev = torch.device("cuda", local)
+    out = {}
+    lib = fb.load()
+    import ctypes
+    for wid in PER_CONFIG:
+        w = workloads.WORKLOADS[wid]
+        q, k, v, k_len = workloads.make_inputs(w)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        kld = None if k_len is None else k_len.to(dev)
+        o = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.float32, device=dev)
+        lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
+        stream = torch.cuda.Stream(device=dev)
+        params = fb.make_params(qd, kd, vd, o, lse, w.causal, w.scale, k_len=kld)
+        pref, sptr = ctypes.byref(params), fb._stream(stream)
+
+        def launch():
+            st = lib.fa_fwd_ex(pref, sptr)
+            if st != fb.FA_OK:
+                raise fb.FaError(st, "fa_fwd_ex")
+
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                launch()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            launch()
+            e1.record(stream)
+        stream.synchronize()
+        est_us = e0.elapsed_time(e1) * 1e3
+        sampler = ClockSampler(local)
+        sampler.start()
+        per, group, reps, total_ms = time_graph_launches(launch, stream, dev, args.steps, PER_CONFIG_MIN_MS, est_us)
+        clocks = sampler.stop()
+        st = percentiles(per)
+        flops = w.flops()
+        peak, _, burst, sustained = tensor_peak(peaks, total_ms)
+        med_s = st["median"] * 1e-3
+        tf = flops / med_s / 1e12
+        entry = {
+            "workload": w.name, "flops": flops,
+            "timing": f"CUDA graph of {group} launches replayed {reps} times; per-launch device time = "
+                      "replay time / launches (CUDA events on the launching stream)",
+            "launches": group * reps, "region_ms": total_ms,
+            "kernel_us": {kk: (vv * 1e3 if isinstance(vv, float) else vv) for kk, vv in st.items()},
+            "tflops": tf, "tflops_p10_time": flops / (st["p10"] * 1e-3) / 1e12,
+            "tflops_p90_time": flops / (st["p90"] * 1e-3) / 1e12,
+            "frac": tf / peak, "frac_of_burst": tf / burst, "frac_of_sustained": tf / sustained,
+            "clocks": clocks,
+        }
+        if clocks and clocks.get("sm_mhz"):
+            cp = clock_peak_tflops(num_sms, clocks["sm_mhz"])
+            entry["clock_peak_tflops"] = cp
+            entry["frac_of_clock_peak"] = tf / cp
+        if k_len is not None:
+            ef = effective_flops(w, k_len.tolist())
+            entry["eff_flops"] = ef
+            entry["eff_tflops"] = ef / med_s / 1e12
+            entry["eff_note"] = "effective FLOPs: 4*d per (query, key) pair with the key inside its length"
+        out[f"w{wid}"] = entry
+        del qd, kd, vd, o, lse, kld
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (the CUDA library has no CPU path)")
@@ -588,8 +739,12 @@ def run_ours(args, world, rank, local):
     peak, peak_label, burst, sustained = tensor_peak(peaks, elapsed_ms, 2.0 if fp8 else 1.0)
     alg_bytes = algorithmic_bytes(w, k_len)
     traffic = measured_traffic(args.workload)
+    dist = percentiles(per_launch)
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
+                "kernel_ms_median": dist["median"], "kernel_ms_p10": dist["p10"], "kernel_ms_p90": dist["p90"],
+                "achieved_at_median": flops / (dist["median"] * 1e-3) / 1e12,
                 "traffic": traffic,
                 "peak_source": f"{peak_src} {peak_label}" + (" x 2 (nominal FP8/BF16 dense ratio)" if fp8 else ""),
                 "kernel": ("fa_fwd_onetile_kernel" if w.d == 256 else "fa_fwd_sm100_kernel")
@@ -597,6 +752,18 @@ def run_ours(args, world, rank, local):
                 "kernel_ms": kernel_ms,
                 "algorithmic_bytes": alg_bytes, "hbm_gbs_algorithmic": alg_bytes / (kernel_ms * 1e-3) / 1e9,
                 "hbm_peak_gbs": float(peaks["hbm_gbs"])}
+    if clocks and clocks.get("sm_mhz"):
+        # the second denominator: SMs x 8192 dense FLOP/clk at the region's median SM clock
+        cp = clock_peak_tflops(num_sms, clocks["sm_mhz"], 2.0 if fp8 else 1.0)
+        roofline["clock_peak_tflops"] = cp
+        roofline["frac_of_clock_peak"] = achieved / cp
+    if k_len is not None:
+        ef = effective_flops(w, k_len.tolist())
+        roofline["eff_flops"] = ef
+        roofline["eff_achieved"] = ef / (kernel_ms * 1e-3) / 1e12
+    per_config = None
+    if not args.no_per_config and world == 1 and args.workload == DEFAULT_WORKLOAD:
+        per_config = measure_per_config(args, local, peaks, num_sms)
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         rate, threads, desc, _ = cpu_oracle_rate(w, q, k, v, k_len, budget_s=15.0)
@@ -613,6 +780,8 @@ def run_ours(args, world, rank, local):
         "gpu_launches": args.steps * (2 if splits > 1 else 1),
         "clocks": clocks,
     }
+    if per_config is not None:
+        line["per_config"] = per_config
     print(json.dumps(line), flush=True)
 
 

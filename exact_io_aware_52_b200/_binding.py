@@ -22,6 +22,7 @@ FA_ERR_UNSUPPORTED = 3
 FA_ERR_CUDA = 4
 FA_ERR_DEVICE_TIMEOUT = 5
 FA_ERR_WORKSPACE_LIMIT = 6
+FA_ERR_SCHED_BUSY = 7
 FA_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024   # include/fa.h
 FA_O_F32 = 0
 FA_O_BF16 = 1
@@ -45,7 +46,7 @@ class FaParams(ctypes.Structure):
         ("flags", ctypes.c_int), ("timeout_ms", ctypes.c_uint32), ("H_kv", ctypes.c_int),
         ("N_k", ctypes.c_int), ("num_splits", ctypes.c_int), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("in_dtype", ctypes.c_int), ("descale_q", ctypes.c_float),
-        ("descale_k", ctypes.c_float), ("descale_v", ctypes.c_float),
+        ("descale_k", ctypes.c_float), ("descale_v", ctypes.c_float), ("test_drop_load", ctypes.c_int),
     ]
 
 
@@ -109,6 +110,10 @@ def load():
             lib.fa_bwd_workspace_bytes.argtypes = [ctypes.POINTER(FaBwdParams)]
             lib.fa_fwd_static_workspace.restype = i
             lib.fa_fwd_static_workspace.argtypes = [ctypes.POINTER(FaParams), ctypes.c_void_p]
+            lib.fa_testhook_sched_next_slot.restype = i
+            lib.fa_testhook_sched_next_slot.argtypes = []
+            lib.fa_testhook_sched_slot.restype = i
+            lib.fa_testhook_sched_slot.argtypes = [i, vp, vp]
             _lib = lib
     return _lib
 
@@ -134,6 +139,8 @@ def load_selftest():
             lib.fa_selftest_mma_e4m3_ts.argtypes = [vp, vp, vp, vp, vp]
             lib.fa_selftest_exp2_poly.restype = i
             lib.fa_selftest_exp2_poly.argtypes = [vp, vp, i, vp]
+            lib.fa_selftest_mma_pair.restype = i
+            lib.fa_selftest_mma_pair.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
             lib.fa_selftest_wait_timeout.restype = i
             lib.fa_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
             _selftest = lib
@@ -175,7 +182,7 @@ def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None):
 
 
 def make_params(q, k, v, o, lse, causal, scale, k_len=None, dev_status=None, flags=0, timeout_ms=0,
-                shape=None, num_splits=0, workspace=None, descale=(0.0, 0.0, 0.0)) -> FaParams:
+                shape=None, num_splits=0, workspace=None, descale=(0.0, 0.0, 0.0), test_drop_load=0) -> FaParams:
     """Fill a fa_fwd_params from tensors (any of them may be None for argument tests).
 
     k, v may be [B, H_kv, N_k, d] with H_kv dividing H and any N_k; workspace is a
@@ -200,7 +207,8 @@ def make_params(q, k, v, o, lse, causal, scale, k_len=None, dev_status=None, fla
                     H_kv=H_kv, N_k=N_k, num_splits=int(num_splits), workspace=_ptr(workspace),
                     workspace_bytes=ws_bytes,
                     in_dtype=FA_IN_E4M3 if getattr(q, "dtype", None) == torch.float8_e4m3fn else FA_IN_BF16,
-                    descale_q=float(descale[0]), descale_k=float(descale[1]), descale_v=float(descale[2]))
+                    descale_q=float(descale[0]), descale_k=float(descale[1]), descale_v=float(descale[2]),
+                    test_drop_load=int(test_drop_load))
 
 
 def workspace_bytes(q, k, num_splits: int) -> int:
@@ -216,13 +224,14 @@ def suggest_splits(q, k) -> int:
 
 
 def fa_fwd_ex(q, k, v, o, lse, causal: bool, scale: float, k_len=None, dev_status=None, flags: int = 0,
-              timeout_ms: int = 0, stream=None, num_splits: int = 0, workspace=None, descale=(0.0, 0.0, 0.0)):
+              timeout_ms: int = 0, stream=None, num_splits: int = 0, workspace=None, descale=(0.0, 0.0, 0.0),
+              test_drop_load: int = 0):
     """fa_fwd_ex: as fa_fwd, plus k_len (int32 [B] CUDA tensor), o may be bf16,
     an optional int32 status word, FA_FLAG_* flags and the wait time limit.
     k and v may be [B, H_kv, N_k, d] (grouped heads, more keys than queries);
     num_splits > 1 splits each row's keys, with `workspace` as scratch."""
     p = make_params(q, k, v, o, lse, causal, scale, k_len, dev_status, flags, timeout_ms,
-                    num_splits=num_splits, workspace=workspace, descale=descale)
+                    num_splits=num_splits, workspace=workspace, descale=descale, test_drop_load=test_drop_load)
     _check(load().fa_fwd_ex(ctypes.byref(p), _stream(stream)), "fa_fwd_ex")
 
 

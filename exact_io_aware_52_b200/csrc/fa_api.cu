@@ -12,10 +12,12 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_internal.h"
 #include "fa_bwd_kernel.cuh"
 #include "fa_combine_kernel.cuh"
 #include "fa_fwd_d256_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
+#include "fa_fwd_pair_kernel.cuh"
 
 namespace {
 
@@ -23,14 +25,22 @@ constexpr int kVersion = 300;  // 0.3.0
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplits = 1024;
 
-// Scheduler words of the forward kernels' dynamic work distribution: one
-// pair per launch slot ([0] next unit, [1] CTAs done), zero at module load
-// and reset to zero by the last CTA of each launch.  A launch takes the next
-// slot round-robin, so up to kSchedSlots launches may be in flight at once
-// on one device (on any streams).
+// Scheduler slots of the dynamic work distribution (causal forward, backward):
+// four words per slot, [0] next unit, [1] CTAs done, [2, 4) the 64-bit owner
+// (grid id + 1 of the launch using the slot, 0: free); zero at module load and
+// returned to zero by the last CTA of each launch.  A launch takes the next
+// slot round-robin; launches that meet on a slot (more than kSchedSlots in
+// flight at once, or one CUDA graph replayed on several streams) serialise on
+// it in the kernel, and a launch whose wait for its slot outlasts its time
+// limit reports FA_ERR_SCHED_BUSY.
 constexpr int kSchedSlots = 64;
-static __device__ uint32_t g_sched[2 * kSchedSlots];
+constexpr int kSchedWords = 4;
+static __device__ __align__(16) uint32_t g_sched[kSchedWords * kSchedSlots];
 std::atomic<uint32_t> g_sched_next{0};
+
+// d = 128 with bf16 inputs on CTA pairs (fa_fwd_pair_kernel.cuh) instead of
+// the one-CTA two-tile kernel.
+constexpr bool kUsePairD128 = false;
 
 struct DeviceInfo {
     bool probed = false;
@@ -38,6 +48,7 @@ struct DeviceInfo {
     int num_sms = 0;
     uint32_t *sched = nullptr;  // g_sched on this device
     bool attr_set[4][2] = {};  // [d = 64, 128, 256, 128 with E4M3 inputs][bf16 out]
+    bool pair_attr_set[2] = {};  // pair kernel [bf16 out]
     bool bwd_attr_set[2] = {};  // backward kernel, [d == 128]
 };
 
@@ -130,8 +141,8 @@ fa_status encode_map_f32(CUtensorMap *map, void *base, int BH, int N, int D) {
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// Validation that needs no device: shared by every entry point.
-fa_status validate(const fa_fwd_params *p) {
+// Validation that needs no device, except the workspace clause.
+fa_status validate_args(const fa_fwd_params *p) {
     if (!p) return FA_ERR_INVALID_ARGUMENT;
     if (p->B < 0 || p->H < 0 || p->N < 0) return FA_ERR_INVALID_ARGUMENT;
     if (!(std::isfinite(p->scale) && p->scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
@@ -143,6 +154,7 @@ fa_status validate(const fa_fwd_params *p) {
     if (p->in_dtype != FA_IN_BF16 && p->in_dtype != FA_IN_E4M3) return FA_ERR_INVALID_ARGUMENT;
     if (!valid_descale(p->descale_q) || !valid_descale(p->descale_k) || !valid_descale(p->descale_v))
         return FA_ERR_INVALID_ARGUMENT;
+    if (p->test_drop_load < 0) return FA_ERR_INVALID_ARGUMENT;
     if (!supported_d(p->d)) return FA_ERR_UNSUPPORTED;
     if (e4m3_in(p) && p->d != 128) return FA_ERR_UNSUPPORTED;
     const long long rows = (long long)p->B * p->H * p->N;
@@ -154,6 +166,13 @@ fa_status validate(const fa_fwd_params *p) {
     if ((reinterpret_cast<uintptr_t>(p->lse) & 3u) || (reinterpret_cast<uintptr_t>(p->k_len) & 3u) ||
         (reinterpret_cast<uintptr_t>(p->dev_status) & 3u))
         return FA_ERR_MISALIGNED;
+    return FA_OK;
+}
+
+// Validation that needs no device: shared by every entry point.
+fa_status validate(const fa_fwd_params *p) {
+    const fa_status st = validate_args(p);
+    if (st != FA_OK || (long long)p->B * p->H * p->N == 0) return st;
     if (p->num_splits > 1) {
         if (!p->workspace || p->workspace_bytes < fa_fwd_workspace_bytes(p)) return FA_ERR_INVALID_ARGUMENT;
         if (!aligned16(p->workspace)) return FA_ERR_MISALIGNED;
@@ -206,6 +225,43 @@ fa_status launch(const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t
         }
     }
     kern<<<grid, threads, smem, stream>>>(kp);
+    return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// d = 128, bf16 inputs, on CTA pairs: a static snake order of units over
+// min(units, SMs / 2) pairs; K is read through a second map whose boxes are
+// one CTA's 64 keys.
+template <bool BF16>
+fa_status launch_pair(const fa::FwdParams &kp, const void *k, int BH_kv, int n_k, DeviceInfo &di, cudaStream_t stream) {
+    fa::PairParams pp;
+    std::memset(&pp, 0, sizeof pp);
+    pp.p = kp;
+    pp.p.dynamic = 0;
+    pp.p.sort_b = 0;
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)128, (cuuint64_t)n_k, (cuuint64_t)BH_kv};
+        cuuint64_t strides[2] = {(cuuint64_t)128 * 2, (cuuint64_t)n_k * 128 * 2};
+        cuuint32_t box[3] = {64, 64, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode(&pp.tm_k64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return FA_ERR_CUDA;
+    }
+    auto kern = fa::fa_fwd_pair_kernel<BF16>;
+    const int smem = fa::pair::PCfg::kSmemBytes;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        bool &set = di.pair_attr_set[BF16];
+        if (!set) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+                return FA_ERR_CUDA;
+            set = true;
+        }
+    }
+    int pairs = di.num_sms / 2;
+    if (pp.p.n_units < pairs) pairs = pp.p.n_units;
+    kern<<<2 * pairs, fa::pair::kThreads, smem, stream>>>(pp);
     return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -281,6 +337,19 @@ fa_status launch_bwd(const fa::bwd::BwdParams &kp, const fa_bwd_params *p, Devic
 
 }  // namespace
 
+namespace fa_detail {
+
+fa_status validate_args(const fa_fwd_params *p) { return ::validate_args(p); }
+
+fa_status probe_current_device() {
+    int dev = 0;
+    DeviceInfo *di = nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    return probe_device(&dev, &di);
+}
+
+}  // namespace fa_detail
+
 extern "C" {
 
 size_t fa_bwd_workspace_bytes(const fa_bwd_params *p) {
@@ -335,7 +404,7 @@ fa_status fa_bwd(const fa_bwd_params *p, void *stream) {
         int band = (di->num_sms + heads_fit - 1) / heads_fit;
         kp.band_tiles = band < 1 ? 1 : (band > kp.n_kv_tiles ? kp.n_kv_tiles : band);
     }
-    kp.sched = di->sched + 2 * (g_sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
+    kp.sched = di->sched + kSchedWords * (g_sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
     kp.causal = p->causal;
     kp.scale = p->scale;
     kp.scale_log2 = (float)((double)p->scale * 1.4426950408889634074);
@@ -403,12 +472,16 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
         const int in_flight = (di->num_sms + sp.splits - 1) / sp.splits;
         int band = (in_flight + heads_fit - 1) / heads_fit;
         kp.band_blocks = band < 1 ? 1 : (band > kp.n_blocks ? kp.n_blocks : band);
-        // causal units differ in cost: hand them out dynamically; equal-cost
-        // (non-causal) units keep the static snake over head-major order
-        kp.dynamic = p->causal ? 1 : 0;
-        if (!kp.dynamic) kp.band_blocks = kp.n_blocks;
+        // causal units differ in cost: hand them out dynamically; key-padded
+        // non-causal units differ by batch element: hand them out dynamically,
+        // batch elements with the most key tiles first (d <= 128, up to
+        // kSortMaxB of them); equal-cost units keep the static snake over
+        // head-major order
+        kp.sort_b = (!p->causal && p->k_len && p->B <= fa::kSortMaxB && p->d <= 128 && sp.splits == 1) ? 1 : 0;
+        kp.dynamic = (p->causal || kp.sort_b) ? 1 : 0;
+        if (!p->causal) kp.band_blocks = kp.n_blocks;
     }
-    kp.sched = di->sched + 2 * (g_sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
+    kp.sched = di->sched + kSchedWords * (g_sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
     kp.causal = p->causal;
     if (e4m3_in(p)) {
         // value scales: Q K^T by descale_q * descale_k (folded into the softmax
@@ -423,10 +496,20 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
         kp.out_scale = 1.f;
     }
     kp.timeout_ns = (uint64_t)(p->timeout_ms ? p->timeout_ms : 2000u) * 1000000ull;
+    kp.drop_load = p->test_drop_load;
 
     const int grid = kp.n_units < di->num_sms ? kp.n_units : di->num_sms;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = p->o_dtype == FA_O_BF16;
+    if (kUsePairD128 && p->d == 128 && !e4m3_in(p) && di->num_sms >= 2) {
+        if (sp.splits > 1) {
+            if ((st = launch_pair<false>(kp, p->k, p->B * H_kv, n_k_map, *di, s)) != FA_OK) return st;
+            return bf16 ? launch_combine_d<true>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)
+                        : launch_combine_d<false>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s);
+        }
+        return bf16 ? launch_pair<true>(kp, p->k, p->B * H_kv, n_k_map, *di, s)
+                    : launch_pair<false>(kp, p->k, p->B * H_kv, n_k_map, *di, s);
+    }
     if (sp.splits > 1) {  // the split pass always writes fp32 partials; the merge writes the output type
         if ((st = launch_d<false>(p->d, e4m3_in(p), kp, *di, grid, s)) != FA_OK) return st;
         return bf16 ? launch_combine_d<true>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)
@@ -534,7 +617,7 @@ fa_status fa_read_device_status(const int32_t *dev_status, void *stream) {
     int32_t h = 0;
     if (cudaMemcpyAsync(&h, dev_status, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess) return FA_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
-    if (h < FA_OK || h > FA_ERR_DEVICE_TIMEOUT) return FA_ERR_CUDA;
+    if (h != FA_OK && h != FA_ERR_DEVICE_TIMEOUT && h != FA_ERR_SCHED_BUSY) return FA_ERR_CUDA;
     return (fa_status)h;
 }
 
@@ -547,10 +630,33 @@ const char *fa_status_string(fa_status s) {
         case FA_ERR_CUDA: return "FA_ERR_CUDA";
         case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
         case FA_ERR_WORKSPACE_LIMIT: return "FA_ERR_WORKSPACE_LIMIT";
+        case FA_ERR_SCHED_BUSY: return "FA_ERR_SCHED_BUSY";
     }
     return "FA_ERR_UNKNOWN";
 }
 
 int fa_version(void) { return kVersion; }
+
+int fa_testhook_sched_next_slot(void) {
+    return (int)(g_sched_next.load(std::memory_order_relaxed) % kSchedSlots);
+}
+
+fa_status fa_testhook_sched_slot(int slot, const uint32_t *set4, uint32_t *get4) {
+    if (slot < 0 || slot >= kSchedSlots) return FA_ERR_INVALID_ARGUMENT;
+    int dev = 0;
+    DeviceInfo *di = nullptr;
+    fa_status st;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        st = probe_device(&dev, &di);
+    }
+    if (st != FA_OK) return st;
+    uint32_t *w = di->sched + kSchedWords * slot;
+    if (set4 && cudaMemcpy(w, set4, kSchedWords * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (get4 && cudaMemcpy(get4, w, kSchedWords * sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FA_ERR_CUDA;
+    return FA_OK;
+}
 
 }  // extern "C"

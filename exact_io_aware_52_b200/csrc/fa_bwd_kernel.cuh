@@ -59,7 +59,7 @@ struct BwdParams {
     int n_kv_tiles;                       // ceil(Nk / 128)
     int n_units;                          // B * H_kv * n_kv_tiles
     int band_tiles;                       // key tiles per band of the unit order (see decode_bunit)
-    uint32_t *sched;                      // this launch's scheduler words: [0] next unit, [1] CTAs done
+    uint32_t *sched;                      // this launch's scheduler slot (as FwdParams::sched)
     int causal;
     float scale;                          // sigma
     float scale_log2;                     // sigma * log2(e)
@@ -87,7 +87,8 @@ struct BCfg {
     static constexpr int kNumBars = 18 + 2 * kUnitQueue;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 4;
-    static constexpr int kOffUnitIds = kOffAbort + 4;          // [kUnitQueue][4] ints
+    static constexpr int kOffClaimed = kOffAbort + 4;          // scheduler slot claimed (int)
+    static constexpr int kOffUnitIds = kOffClaimed + 4;        // [kUnitQueue][4] ints
     // + slack to align the base to 1024 bytes; at least 117 KB so that one CTA
     // (which allocates all of TMEM) runs per SM
     static constexpr int kSmemBytes =
@@ -502,11 +503,11 @@ __device__ __forceinline__ void load_role(const BwdParams &p, uint64_t *bars, vo
     }
     if (!ok) record_timeout_b(p);
     // drain: every copy this thread issued has landed before the CTA may exit
-    if (gkv > 0) mbar_wait_drain(&bars[C::kBarKV], (gkv - 1) & 1, to);
+    if (gkv > 0) mbar_wait_drain(&bars[C::kBarKV], (gkv - 1) & 1);
     const uint32_t n = gt < 2u ? gt : 2u;
     for (uint32_t i = 0; i < n; ++i) {
         const uint32_t g = gt - 1 - i;
-        mbar_wait_drain(&bars[C::kBarSlot + (g & 1)], (g >> 1) & 1, to);
+        mbar_wait_drain(&bars[C::kBarSlot + (g & 1)], (g >> 1) & 1);
     }
 }
 
@@ -540,6 +541,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1) fa_bwd_sm100_kernel(const __
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffAbort);
+    volatile int *claimed = reinterpret_cast<volatile int *>(smem + C::kOffClaimed);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const UnitQueue uq{reinterpret_cast<volatile int *>(smem + C::kOffUnitIds), &bars[C::kBarUnitFull],
@@ -554,6 +556,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1) fa_bwd_sm100_kernel(const __
             mbar_init(&bars[i], unit_free ? 130u : (per_row ? 128u : 1u));
         }
         *abort_flag = 0;
+        *claimed = sched_claim(p.sched, p.timeout_ns) ? 1 : 0;
         fence_mbar_init();
     }
     if (warp == bwd::kMmaWarp) {
@@ -564,13 +567,18 @@ __global__ void __launch_bounds__(bwd::kThreads, 1) fa_bwd_sm100_kernel(const __
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (!*claimed) {  // the scheduler slot stayed in use by another launch: no work, report it
+        if (threadIdx.x == 0) record_status(p.status, kStatusSchedBusy);
+        if (warp == bwd::kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+        return;
+    }
     if (warp < 4) {
         if (!bwd::compute_role<D>(p, bars, abort_flag, uq, tmem, smem, warp, lane)) bwd::record_timeout_b(p);
     } else if (warp == bwd::kMmaWarp) {
         if (lane == 0) {
             if (!bwd::mma_role<D>(p, bars, abort_flag, uq, tmem, smem_u32(smem))) bwd::record_timeout_b(p);
             tc_commit(&bars[C::kBarDrain]);
-            mbar_wait_drain(&bars[C::kBarDrain], 0, p.timeout_ns);
+            mbar_wait_drain(&bars[C::kBarDrain], 0);
         }
     } else if (warp == bwd::kLoadWarp) {
         if (lane == 0) bwd::load_role<D>(p, bars, abort_flag, uq, smem);

@@ -78,7 +78,8 @@ struct Cfg1 {
     static constexpr int kNumBars = kBarDrain + 1;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 4;
-    static constexpr int kOffUnitIds = kOffAbort + 4;
+    static constexpr int kOffClaimed = kOffAbort + 4;  // scheduler slot claimed (int)
+    static constexpr int kOffUnitIds = kOffClaimed + 4;
     static constexpr int kSmemUsed = kOffUnitIds + 16 * kUnitQueue;
     static constexpr int kSmemBytes = kSmemUsed + 1024;  // + slack to align the base to 1024 bytes
     static_assert(kHalfBytes % 1024 == 0 && kBlockBytes % 1024 == 0, "1024-byte alignment of swizzled tiles");
@@ -129,7 +130,6 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
     using C = Cfg1<D>;
     const int row_in_tile = warp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const float LN2 = 0.69314718055994530942f;
     const float NEG_INF = __int_as_float(0xff800000);
     const uint32_t t_o = tmem + lane_off + kColO;
     const uint64_t to = p.timeout_ns;
@@ -154,9 +154,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         if (p.k_len) lim = min(max(__ldg(p.k_len + u.b), 0), p.Nk);
         if (p.causal) lim = min(lim, row + 1 + (p.Nk - p.N));
 
-        float m_ref = 0.f;  // reference maximum, log2 units
-        float l = 0.f;      // running sum of 2^(x - m_ref), unrounded: gives lse
-        float lr = 0.f;     // running sum of the bf16-rounded terms: O's normaliser
+        RowState st;
         for (int j = 0; j < n; ++j, ++gs) {
             const uint32_t buf = gs & 1;
             const uint32_t t_s = tmem + lane_off + buf * 128u;
@@ -165,36 +163,13 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             if (!ok) break;
             tc_fence_after();
 
-            const int kv0 = (u.lo + j) * BN;
-            const bool masked = kv0 + BN > lim;
             float s[BN];
             uint32_t pk0[32], pk1[32];
             float2 ls = make_float2(0.f, 0.f);
-            float lrs = 0.f;
-            tmem_ld32f(t_s + 0, s);
-            tmem_ld32f(t_s + 32, s + 32);
-            tmem_ld32f(t_s + 64, s + 64);
-            tmem_ld32f(t_s + 96, s + 96);
-            tmem_ld_wait();
-            tmem_reg_fence_f<BN>(s);
-            if (masked) {
-                mask_scores<0>(s, kv0, lim);
-                mask_scores<1>(s, kv0, lim);
-            }
-            const float m_new = fmaxf(max64(s), max64(s + 64)) * p.scale_log2;
-            float alpha = 1.f;
-            bool resc = false;
-            if (j == 0) {
-                m_ref = (m_new == NEG_INF) ? 0.f : m_new;
-                l = 0.f;
-                lr = 0.f;
-            } else if (m_new > m_ref + p.tau) {
-                alpha = ex2_approx(m_ref - m_new);
-                l *= alpha;
-                lr *= alpha;
-                m_ref = m_new;
-                resc = true;
-            }
+            load_score_row(t_s, s);
+            const float m_new = masked_row_max(s, (u.lo + j) * BN, lim, p.scale_log2);
+            float alpha;
+            const bool resc = update_reference(st, j, m_new, p.tau, alpha);
             // the products before this tile's predecessor are complete (the
             // commit behind S ready covers them): consume their phases
             const bool any_resc = __any_sync(0xffffffffu, resc);
@@ -203,38 +178,17 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             if (!ok) break;
             if (any_resc) {
                 tc_fence_after();
-#pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
-                    uint32_t r[32];
-                    tmem_ld32(t_o + ch * 32, r);
-                    tmem_ld_wait();
-                    tmem_reg_fence(r);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-                    tmem_st32(t_o + ch * 32, r);
-                }
+                rescale_o_row<D>(t_o, alpha);
             }
-            if constexpr (kLateSums) {
-                exp_half_p<0>(s, p.scale_log2, -m_ref, pk0, ls);
-                tmem_st32(t_s + 0, pk0);
-                exp_half_p<1>(s, p.scale_log2, -m_ref, pk1, ls);
-                tmem_st32(t_s + 32, pk1);
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&bars[C::kBarPFull + buf]);
-                l += ls.x + ls.y;
-                lr += rounded_sum(pk0, pk1);
-            } else {
-                exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
-                tmem_st32(t_s + 0, pk0);
-                exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
-                tmem_st32(t_s + 32, pk1);
-                l += ls.x + ls.y;
-                lr += lrs;
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&bars[C::kBarPFull + buf]);
-            }
+            exp_half_p<0>(s, p.scale_log2, -st.m_ref, pk0, ls);
+            tmem_st32(t_s + 0, pk0);
+            exp_half_p<1>(s, p.scale_log2, -st.m_ref, pk1, ls);
+            tmem_st32(t_s + 32, pk1);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars[C::kBarPFull + buf]);
+            st.l += ls.x + ls.y;
+            st.lr += rounded_sum(pk0, pk1);
         }
         if (ok) {
             ok = wait_pv_upto<D>(bars, waited, (long long)gs - 1, abort_flag, to);
@@ -245,17 +199,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             break;
         }
         tc_fence_after();
-        const bool empty = !(lr > 0.f);
-        const float inv_l = empty ? 0.f : 1.f / lr;
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t r[32];
-            tmem_ld32(t_o + ch * 32, r);
-            tmem_ld_wait();
-            tmem_reg_fence(r);
-            if (row_valid) store_row_chunk<D, O_BF16>(p.o, row_id, ch, r, inv_l);
-        }
-        if (row_valid) p.lse[row_id] = empty ? NEG_INF : (m_ref + log2f(l)) * LN2;
+        write_row<D, O_BF16>(t_o, p.o, p.lse, row_id, row_valid, st.lr, 1.f, st.m_ref + log2f(st.l));
         tc_fence_before();
         mbar_arrive(&bars[C::kBarOFree]);
         ++tl;
@@ -363,6 +307,8 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
     prefetch_tensormap(&p.tm_v);
     const uint64_t to = p.timeout_ns;
     uint32_t tq = 0, g = 0;
+    // test only: the ring load this CTA never issues (its ring position), or none
+    const uint32_t drop = (blockIdx.x == 0 && p.drop_load > 0) ? (uint32_t)(p.drop_load - 1) : 0xFFFFFFFFu;
     bool ok = true;
     // key tile `kt` of K or V as D / 128 half tiles (d columns [128 h, 128 h + 128))
     auto load_tile = [&](const CUtensorMap *map, int kt, int bh_kv) -> bool {
@@ -370,11 +316,13 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
         for (int h = 0; h < C::kHalves; ++h) {
             const uint32_t slot = g % C::kSlots, round = g / C::kSlots;
             if (round > 0 && !mbar_wait(&bars[C::kBarEmpty + slot], (round - 1) & 1, abort_flag, to)) return false;
-            mbar_arrive_expect_tx(&bars[C::kBarFull + slot], kHalfBytes);
+            if (g != drop) {
+                mbar_arrive_expect_tx(&bars[C::kBarFull + slot], kHalfBytes);
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-                tma_load_3d(ring + slot * kHalfBytes + c * kBlockBytes, map, &bars[C::kBarFull + slot], h * 128 + c * 64,
-                            kt * BN, bh_kv);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_3d(ring + slot * kHalfBytes + c * kBlockBytes, map, &bars[C::kBarFull + slot],
+                                h * 128 + c * 64, kt * BN, bh_kv);
+            }
             ++g;
         }
         return true;
@@ -409,11 +357,11 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
     }
     if (!ok) record_timeout(p);
     // drain: every copy this thread issued has landed before the CTA may exit
-    if (tq > 0) mbar_wait_drain(&bars[C::kBarQFull], (tq - 1) & 1, to);
+    if (tq > 0) mbar_wait_drain(&bars[C::kBarQFull], (tq - 1) & 1);
     const uint32_t nr = g < (uint32_t)C::kSlots ? g : (uint32_t)C::kSlots;
     for (uint32_t i = 0; i < nr; ++i) {
         const uint32_t gi = g - 1 - i;
-        mbar_wait_drain(&bars[C::kBarFull + gi % C::kSlots], (gi / C::kSlots) & 1, to);
+        if (gi != drop) mbar_wait_drain(&bars[C::kBarFull + gi % C::kSlots], (gi / C::kSlots) & 1);
     }
 }
 
@@ -430,6 +378,7 @@ __global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_onetile_kernel(const
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffAbort);
+    volatile int *claimed = reinterpret_cast<volatile int *>(smem + C::kOffClaimed);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -442,6 +391,7 @@ __global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_onetile_kernel(const
             mbar_init(&bars[i], unit_free ? 129u : (per_row ? 128u : 1u));
         }
         *abort_flag = 0;
+        *claimed = p.dynamic ? (sched_claim(p.sched, p.timeout_ns) ? 1 : 0) : 1;
         fence_mbar_init();
     }
     if (warp == d256::kMmaWarp) {
@@ -452,6 +402,11 @@ __global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_onetile_kernel(const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (!*claimed) {  // the scheduler slot stayed in use by another launch: no work, report it
+        if (threadIdx.x == 0) record_status(p.status, kStatusSchedBusy);
+        if (warp == d256::kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+        return;
+    }
 
     if (warp < d256::kSoftmaxWarps) {
         if (!d256::softmax_role<D, O_BF16>(p, bars, abort_flag, uq, tmem, warp, lane)) record_timeout(p);
@@ -459,7 +414,7 @@ __global__ void __launch_bounds__(d256::kThreads, 1) fa_fwd_onetile_kernel(const
         if (lane == 0) {
             if (!d256::mma_role<D>(p, bars, abort_flag, uq, tmem, smem_u32(sQ), smem_u32(ring))) record_timeout(p);
             tc_commit(&bars[C::kBarDrain]);
-            mbar_wait_drain(&bars[C::kBarDrain], 0, p.timeout_ns);
+            mbar_wait_drain(&bars[C::kBarDrain], 0);
         }
     } else if (warp == d256::kLoadWarp) {
         if (lane == 0) d256::load_role<D>(p, bars, abort_flag, uq, sQ, ring);

@@ -46,12 +46,10 @@
 // drains its in-flight copies and MMAs (again bounded), frees TMEM and exits.
 #pragma once
 
-#include "sm100_ptx.cuh"
+#include "fa_softmax_row.cuh"
 
 namespace fa {
 
-constexpr int BM = 128;        // query rows per tile (tcgen05 M)
-constexpr int BN = 128;        // keys per tile
 constexpr int kQTiles = 2;     // query tiles per work unit
 constexpr int kUnitRows = BM * kQTiles;
 constexpr int kSoftmaxWarps = 8;
@@ -67,32 +65,20 @@ constexpr int kControlRegs = 56;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kUnitQueue = 4;  // depth of the shared-memory queue of work-unit ids
-constexpr int kStatusTimeout = 5;  // FA_ERR_DEVICE_TIMEOUT
-// Of every kPolyPeriod key pairs of a score row, the last kPolyPairs take
-// their exponentials from the FMA-pipe polynomial, the rest from MUFU ex2.
-// Measured on workload 4 (B200, 300 launches): 0 of 4 -> 2.30 ms, 1 of 4 ->
-// 2.44 ms, 2 of 4 -> 2.49 ms: the softmax is not MUFU-throughput bound here,
-// so the polynomial's extra instructions only cost; it stays off.
-constexpr int kPolyPeriod = 4;
-constexpr int kPolyPairs = 0;
-// P to bf16: round to nearest even (cvt) when false; truncation (keep the
-// high half of each fp32 word, one byte permute per pair) when true.
-constexpr bool kPackTruncate = false;
-// The tile's sum of the bf16-rounded probabilities (two mixed-precision adds
-// per pair) is taken after "P ready", from the packed pairs, instead of
-// between the exponentials, so that the tensor core gets P sooner; the
-// unrounded sum (one packed add per pair) stays beside the exponentials.
-constexpr bool kLateSums = true;
-static_assert(!kLateSums || (kPolyPairs == 0 && !kPackTruncate), "late sums: MUFU exponentials, rounded P");
-// P V in two halves of 64 keys: the softmax releases P for keys [0, 64) as
-// soon as it is in TMEM, so the tensor core multiplies that half while the
-// softmax computes the other, and only P V for keys [64, 128) plus the next
-// Q K^T remain between "P ready" and the next "S ready".  Measured on B200
-// (300 launches each): d = 64 (B8 H12 N1024 causal) 48.5 -> 47.1 us; d = 128
-// (B1 H32 N16384 causal) 2.249 -> 2.306 ms, where the extra store wait in the
-// middle of the softmax costs more than the overlap gains.  On for d = 64 only.
+// Largest batch for which the unit order sorts the batch elements by their key
+// tiles (a table of this many ints in shared memory).
+constexpr int kSortMaxB = 128;
+constexpr int kStatusTimeout = 5;    // FA_ERR_DEVICE_TIMEOUT
+constexpr int kStatusSchedBusy = 7;  // FA_ERR_SCHED_BUSY
+// Separate P columns (d = 64): O_A and O_B take 64 TMEM columns each, which
+// leaves 128 columns for P_A [384, 448) and P_B [448, 512).  P then no longer
+// overwrites S, so Q_X K_{j+1}^T may run as soon as the softmax has read
+// S_X(j) (barrier s_free) instead of after P_X V_j: the softmax of a tile no
+// longer waits for the P V -> Q K^T chain of its own previous tile.  The
+// price: a rescale of O_X and the store of P_X(j+1) first wait for P_X V_j
+// (barrier pv_done, one phase per product).
 template <int D>
-constexpr bool kSplitPV = (D == 64);
+constexpr bool kSepP = (D == 64);
 // The V ring slot of key tile j-1 is released right after the last P_X V_{j-1}
 // product is issued (before Q_B K_j^T) instead of at the end of the step.
 // Measured on B200 (300 launches): E4M3 (B1 H32 N16384 causal) 1.852 ->
@@ -103,6 +89,7 @@ constexpr bool kEarlyVRelease = F8;
 
 __device__ __forceinline__ uint32_t col_s(uint32_t x) { return x * 128u; }                  // S_X, P_X
 __device__ __forceinline__ uint32_t col_o(uint32_t x, uint32_t d) { return 256u + x * d; }  // O_X
+__device__ __forceinline__ uint32_t col_p_sep(uint32_t x) { return 384u + x * 64u; }         // P_X (d = 64)
 
 struct FwdParams {
     CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps over [B*H][N][D] (Q) and [B*H_kv][Nk][D] (K, V) bf16;
@@ -121,12 +108,18 @@ struct FwdParams {
     int n_units;                   // B * H * n_blocks * n_splits
     int band_blocks;               // query blocks per band of the unit order (see decode_unit)
     int dynamic;                   // units handed out by the counter (1) or in the static snake order (0)
-    uint32_t *sched;               // this launch's scheduler words: [0] next unit, [1] CTAs done
+    int sort_b;                    // 1: key-padded non-causal units go batch element by batch element,
+                                   // most key tiles first (B <= kSortMaxB; dynamic)
+    uint32_t *sched;               // this launch's scheduler slot: [0] next unit, [1] CTAs done,
+                                   // [2, 4) owner (64-bit grid id + 1 of the launch using it, 0: free)
     int causal;
     float scale_log2;              // scale * log2(e)
     float tau;                     // rescale threshold in log2 units (<= 0: rescale on any growth)
     float out_scale;               // factor on O (the value scale of E4M3 inputs; 1 for bf16)
     uint64_t timeout_ns;
+    int drop_load;                 // test only (0: off): CTA 0's TMA producer never issues its
+                                   // drop_load-th K-tile load (d = 256: ring load), so the
+                                   // wait for it runs out and the time-out path runs
 };
 
 // F8: Q, K and V in E4M3 (one byte per element, d = 128 only), products on
@@ -156,17 +149,24 @@ struct Cfg {
     static constexpr int kBarPFull = kBarSFull + 2;          // [2]
     static constexpr int kBarOFinal = kBarPFull + 2;         // [2]
     static constexpr int kBarOFree = kBarOFinal + 2;         // [2]
-    static constexpr int kBarPHalf = kBarOFree + 2;          // [2] P of keys [0, 64) in TMEM
-    static constexpr int kBarUnitFull = kBarPHalf + 2;       // [kUnitQueue]
+    static constexpr int kBarSFree = kBarOFree + 2;          // [2] S_X read by the softmax (separate P)
+    static constexpr int kBarPvDone = kBarSFree + 2;         // [2] P_X V complete (separate P)
+    static constexpr int kBarUnitFull = kBarPvDone + 2;      // [kUnitQueue]
     static constexpr int kBarUnitFree = kBarUnitFull + kUnitQueue;  // [kUnitQueue]
     static constexpr int kBarDrain = kBarUnitFree + kUnitQueue;
     static constexpr int kNumBars = kBarDrain + 1;
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 4;
-    static constexpr int kOffUnitIds = kOffAbort + 4;                // [kUnitQueue][4] ints
-    static constexpr int kSmemUsed = kOffUnitIds + 16 * kUnitQueue;
+    static constexpr int kOffClaimed = kOffAbort + 4;                // scheduler slot claimed (int)
+    static constexpr int kOffUnitIds = kOffClaimed + 4;              // [kUnitQueue][4] ints
+    static constexpr int kOffBOrder = kOffUnitIds + 16 * kUnitQueue;  // [kSortMaxB] ints
+    // d = 64: per softmax warp a [32][36]-float stage for coalesced O stores
+    static constexpr bool kStageO = kSepP<D> && !F8;
+    static constexpr int kOffStage = (kOffBOrder + 4 * kSortMaxB + 127) & ~127;  // float4 accesses
+    static constexpr int kSmemUsed = kOffStage + (kStageO ? kSoftmaxWarps * 32 * 36 * 4 : 0);
     static constexpr int kSmemBytes = kSmemUsed + 1024;  // + slack to align the base to 1024 bytes
     static_assert(kChunkBytes % 1024 == 0 && kTileBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
+    static_assert(kOffStage % 16 == 0, "the O stage is accessed as float4");
     static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
     static_assert(2 * kSmemBytes > 233472, "one CTA per SM: TMEM is allocated whole");
 };
@@ -196,7 +196,9 @@ struct UnitQueue {
     volatile int *ids;  // [kUnitQueue][4]: unit id, then two words the producer may attach
     uint64_t *full;     // [kUnitQueue], one arrival: the producer has written the entry
     uint64_t *free;     // [kUnitQueue], one arrival per consuming thread
+    const int *b_order; // batch elements longest first (FwdParams::sort_b), else nullptr
 };
+
 
 // Producer (one thread), step 1: the id of this CTA's k-th unit, or -1 when
 // none is left (ok turns false when the wait for a free entry times out).
@@ -253,14 +255,49 @@ __device__ __forceinline__ int unit_pop(const UnitQueue &q, int k, volatile int 
     return t;
 }
 
+// Scheduler slots are shared by all launches on a device (taken round-robin
+// by the host), so two launches in flight at once may meet on one slot (more
+// launches in flight than slots, or one CUDA graph replayed on several
+// streams).  Every CTA therefore claims the slot for its grid before it takes
+// a unit: the owner word holds the grid id + 1 of the launch using the slot
+// (0: free), set by the first CTA of the launch to arrive and cleared by the
+// last to leave.  A CTA that finds another launch's grid id there waits,
+// bounded in wall time; the launches serialise on the slot instead of
+// sharing its counter.  Returns false when the limit passes (the CTA then
+// skips its work and reports FA_ERR_SCHED_BUSY).
+__device__ __forceinline__ bool sched_claim(uint32_t *sched, uint64_t timeout_ns) {
+    unsigned long long *owner = reinterpret_cast<unsigned long long *>(sched + 2);
+    const unsigned long long me = grid_id() + 1ull;
+    uint64_t t0 = 0;
+    for (;;) {
+        const unsigned long long old = atomicCAS(owner, 0ull, me);
+        if (old == 0ull || old == me) {
+            __threadfence();
+            return true;
+        }
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > timeout_ns) return false;
+        __nanosleep(1000);
+    }
+}
+
 // The last CTA to finish resets the launch's scheduler words for the next
-// launch that uses them (every CTA has taken its last id by then).
+// launch that uses them (every CTA has taken its last id by then), and only
+// then frees the slot.
 __device__ __forceinline__ void sched_release(uint32_t *sched) {
     __threadfence();
     if (atomicAdd(sched + 1, 1u) == gridDim.x - 1) {
         atomicExch(sched, 0u);
         atomicExch(sched + 1, 0u);
+        __threadfence();
+        atomicExch(reinterpret_cast<unsigned long long *>(sched + 2), 0ull);
     }
+}
+
+// Stores `code` in the optional status word unless an earlier error is there.
+__device__ __forceinline__ void record_status(int32_t *status, int code) {
+    if (status) atomicCAS(reinterpret_cast<int *>(status), 0, code);
 }
 
 // Unit numbering: the query blocks of every (b, h) are cut into bands of
@@ -280,11 +317,16 @@ __device__ __forceinline__ void band_decode(const FwdParams &p, int r, int &bh, 
     blk = p.n_blocks - 1 - (band * p.band_blocks + (in_band - bh * bsz));
 }
 
-__device__ __forceinline__ UnitCoord decode_unit(const FwdParams &p, int t) {
+__device__ __forceinline__ UnitCoord decode_unit(const FwdParams &p, int t, const int *b_order) {
     UnitCoord u;
     u.split = t % p.n_splits;
     band_decode(p, t / p.n_splits, u.bh, u.blk);
     u.b = u.bh / p.H;
+    if (b_order) {  // batch elements with more key tiles first
+        const int h = u.bh - u.b * p.H;
+        u.b = b_order[u.b];
+        u.bh = u.b * p.H + h;
+    }
     u.bh_kv = u.b * p.H_kv + (u.bh - u.b * p.H) / p.group;
     u.lo = u.split * p.split_tiles;
     int kv_lim = p.Nk;
@@ -305,153 +347,14 @@ __device__ __forceinline__ void record_timeout(const FwdParams &p) {
     if (p.status) atomicCAS(reinterpret_cast<int *>(p.status), 0, kStatusTimeout);
 }
 
-// Bounded wait that ignores the abort flag: used to drain in-flight work.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t timeout_ns) {
+// Bounded wait that ignores the abort flag: used to drain in-flight work (TMA
+// copies and MMAs that were issued and will complete within microseconds).
+// Its limit is fixed and generous, independent of the caller's time limit,
+// so that a short timeout_ms never lets a CTA exit with copies in flight.
+constexpr uint64_t kDrainTimeoutNs = 1000000000ull;
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     int dummy = 0;
-    return mbar_wait(bar, parity, &dummy, timeout_ns);
-}
-
-template <int D, bool O_BF16>
-__device__ __forceinline__ void store_row_chunk(void *o, size_t row_id, int ch, const uint32_t (&r)[32], float inv_l) {
-    if constexpr (O_BF16) {
-        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(o) + row_id * D + ch * 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l);
-            v.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l);
-            v.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l);
-            v.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l);
-            dst[i] = v;
-        }
-    } else {
-        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(o) + row_id * D + ch * 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(r[4 * i + 0]) * inv_l, __uint_as_float(r[4 * i + 1]) * inv_l,
-                                 __uint_as_float(r[4 * i + 2]) * inv_l, __uint_as_float(r[4 * i + 3]) * inv_l);
-    }
-}
-
-// Fills one output row with a constant (0 for rows without allowed keys, NaN
-// for rows of a unit abandoned after a time-out) and sets its lse.
-template <int D, bool O_BF16>
-__device__ __forceinline__ void fill_row(void *o, float *lse, size_t row_id, bool nan, float lv) {
-    if constexpr (O_BF16) {
-        const uint16_t b = nan ? 0x7fc0 : 0;
-        uint16_t *dst = reinterpret_cast<uint16_t *>(o) + row_id * D;
-        for (int i = 0; i < D; ++i) dst[i] = b;
-    } else {
-        const float f = nan ? __int_as_float(0x7fc00000) : 0.f;
-        float *dst = reinterpret_cast<float *>(o) + row_id * D;
-        for (int i = 0; i < D; ++i) dst[i] = f;
-    }
-    lse[row_id] = lv;
-}
-
-// max of 64 scores: four chains of three-input maxima
-__device__ __forceinline__ float max64(const float *v) {
-    float a0 = fmaxf(v[0], v[1]), a1 = fmaxf(v[2], v[3]), a2 = fmaxf(v[4], v[5]), a3 = fmaxf(v[6], v[7]);
-#pragma unroll
-    for (int c = 8; c < 64; c += 8) {
-        a0 = fmax3(a0, v[c], v[c + 1]);
-        a1 = fmax3(a1, v[c + 2], v[c + 3]);
-        a2 = fmax3(a2, v[c + 4], v[c + 5]);
-        a3 = fmax3(a3, v[c + 6], v[c + 7]);
-    }
-    return fmaxf(fmax3(a0, a1, a2), a3);
-}
-
-// Masking step for keys [64H, 64H+64) of a tile starting at key kv0: keys at
-// or beyond the row's limit get -inf.
-template <int H>
-__device__ __forceinline__ void mask_scores(float *s, int kv0, int lim) {
-#pragma unroll
-    for (int c = 64 * H; c < 64 * H + 64; ++c)
-        if (kv0 + c >= lim) s[c] = __int_as_float(0xff800000);
-}
-
-// Probabilities of keys [64H, 64H+64) of one score row against reference -neg_m
-// (log2 units): p = 2^(s * scale_log2 - m), summed unrounded into `ls` and as
-// the bf16 values the tensor core will use into `lrs`, and packed as bf16
-// pairs into pk (column c holds keys 64H + 2c and 64H + 2c + 1).
-template <int H>
-__device__ __forceinline__ void exp_half(const float *s, float scale_log2, float neg_m, uint32_t (&pk)[32],
-                                         float2 &ls, float &lrs) {
-    const float2 sl2 = make_float2(scale_log2, scale_log2);
-    const float2 nm = make_float2(neg_m, neg_m);
-    float2 a[4] = {ls, make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-    float b[4] = {lrs, 0.f, 0.f, 0.f};
-    float2 b2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-    for (int c = 0; c < 64; c += 2) {
-        const float2 xx = __ffma2_rn(make_float2(s[64 * H + c], s[64 * H + c + 1]), sl2, nm);
-        const bool poly = ((c >> 1) % kPolyPeriod) >= kPolyPeriod - kPolyPairs;
-        const float2 pp = poly ? exp2_poly2(xx) : make_float2(ex2_approx(xx.x), ex2_approx(xx.y));
-        a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], pp);
-        uint32_t pb;
-        if constexpr (kPackTruncate) {
-            pb = __byte_perm(__float_as_uint(pp.x), __float_as_uint(pp.y), 0x7632);
-            b2[(c >> 1) & 3] = __fadd2_rn(b2[(c >> 1) & 3], make_float2(__uint_as_float(pb << 16),
-                                                                        __uint_as_float(pb & 0xFFFF0000u)));
-        } else {
-            pb = pack_bf16x2(pp.x, pp.y);
-            b[(c >> 1) & 3] = add_bf16x2_to(b[(c >> 1) & 3], pb);
-        }
-        pk[c >> 1] = pb;
-    }
-    ls = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
-    const float2 bb = __fadd2_rn(__fadd2_rn(b2[0], b2[1]), __fadd2_rn(b2[2], b2[3]));
-    lrs = ((b[0] + b[1]) + (b[2] + b[3])) + (bb.x + bb.y);
-}
-
-// Probabilities of keys [64H, 64H+64) as in exp_half, without the rounded
-// sum: pk holds the bf16 pairs, `ls` gains the unrounded values.
-template <int H>
-__device__ __forceinline__ void exp_half_p(const float *s, float scale_log2, float neg_m, uint32_t (&pk)[32],
-                                           float2 &ls) {
-    const float2 sl2 = make_float2(scale_log2, scale_log2);
-    const float2 nm = make_float2(neg_m, neg_m);
-    float2 a[4] = {ls, make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-    for (int c = 0; c < 64; c += 2) {
-        const float2 xx = __ffma2_rn(make_float2(s[64 * H + c], s[64 * H + c + 1]), sl2, nm);
-        const float2 pp = make_float2(ex2_approx(xx.x), ex2_approx(xx.y));
-        a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], pp);
-        pk[c >> 1] = pack_bf16x2(pp.x, pp.y);
-    }
-    ls = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
-}
-
-// Sum of a tile's 128 bf16 probabilities (two per word of pk0 and pk1).
-__device__ __forceinline__ float rounded_sum(const uint32_t (&pk0)[32], const uint32_t (&pk1)[32]) {
-    float b[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        b[i & 3] = add_bf16x2_to(b[i & 3], pk0[i]);
-        b[(i + 2) & 3] = add_bf16x2_to(b[(i + 2) & 3], pk1[i]);
-    }
-    return (b[0] + b[1]) + (b[2] + b[3]);
-}
-
-// E4M3 probabilities of one 128-key score row: p = 2^(s * scale_log2 - m)
-// summed unrounded into `ls` and rounded to E4M3, four keys per 32-bit
-// column (key 4c + i in byte i of column c).
-__device__ __forceinline__ void exp_e4m3(const float *s, float scale_log2, float neg_m, uint32_t (&pk)[32],
-                                         float2 &ls) {
-    const float2 sl2 = make_float2(scale_log2, scale_log2);
-    const float2 nm = make_float2(neg_m, neg_m);
-    float2 a[4] = {ls, make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-    for (int c = 0; c < 128; c += 4) {
-        const float2 x0 = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2, nm);
-        const float2 x1 = __ffma2_rn(make_float2(s[c + 2], s[c + 3]), sl2, nm);
-        const float2 p0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
-        const float2 p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
-        a[(c >> 2) & 3] = __fadd2_rn(a[(c >> 2) & 3], __fadd2_rn(p0, p1));
-        pk[c >> 2] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
-    }
-    ls = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+    return mbar_wait(bar, parity, &dummy, kDrainTimeoutNs);
 }
 
 // ------------------------------------------------------------------ softmax
@@ -463,27 +366,40 @@ constexpr float kF8Shift = 8.f;
 
 template <int D, bool O_BF16, bool F8>
 __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
-                                             const UnitQueue &uq, uint32_t tmem, int x, int warp, int lane) {
+                                             const UnitQueue &uq, uint32_t tmem, int x, int warp, int lane,
+                                             float *stage) {
     using C = Cfg<D, F8>;
     const int row_in_tile = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const float LN2 = 0.69314718055994530942f;
     const float NEG_INF = __int_as_float(0xff800000);
     uint64_t *s_full = &bars[C::kBarSFull + x];
     uint64_t *p_full = &bars[C::kBarPFull + x];
-    uint64_t *p_half = &bars[C::kBarPHalf + x];
     uint64_t *o_final = &bars[C::kBarOFinal + x];
     uint64_t *o_free = &bars[C::kBarOFree + x];
+    uint64_t *s_free = &bars[C::kBarSFree + x];
+    uint64_t *pv_done = &bars[C::kBarPvDone + x];
+    constexpr bool kSep = kSepP<D> && !F8;
     const uint32_t t_s = tmem + lane_off + col_s(x);
     const uint32_t t_o = tmem + lane_off + col_o(x, D);
+    const uint32_t t_p = tmem + lane_off + (kSep ? col_p_sep(x) : col_s(x));
     uint32_t gs = 0;  // S tiles of this query tile consumed so far (s_full / p_full phase)
     uint32_t tl = 0;  // units in which this query tile had work (o_final / o_free phase)
+    uint32_t pv_known = 0;  // separate P: P_X V products known to be complete
+    // separate P: wait until the first n P_X V products are complete (phases
+    // complete in order, and product n cannot start before this thread stores
+    // P_X(n), so the parity of phase n - 1 is unambiguous)
+    auto ensure_pv = [&](uint32_t n) -> bool {
+        if (pv_known >= n) return true;
+        const bool w = mbar_wait(pv_done, (n - 1) & 1, abort_flag, p.timeout_ns);
+        pv_known = n;
+        return __all_sync(0xffffffffu, w);
+    };
     bool ok = true;
     for (int k = 0; ok; ++k) {
         const int t = p.dynamic ? unit_pop(uq, k, abort_flag, p.timeout_ns, ok) : unit_static(p, k);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok || t < 0) break;
-        const UnitCoord u = decode_unit(p, t);
+        const UnitCoord u = decode_unit(p, t, uq.b_order);
         const int row = u.blk * kUnitRows + x * BM + row_in_tile;
         const bool row_valid = row < p.N;
         // output row: [split][B*H][N] (the split index is 0 without key splits)
@@ -497,104 +413,69 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         if (p.k_len) lim = min(max(__ldg(p.k_len + u.b), 0), p.Nk);
         if (p.causal) lim = min(lim, row + 1 + (p.Nk - p.N));
 
-        float m_ref = 0.f;  // reference maximum, log2 units
-        float l = 0.f;      // running sum of 2^(x - m_ref), unrounded: gives lse
-        float lr = 0.f;     // running sum of bf16(2^(x - m_ref)), the weights the tensor core
-                            // multiplies V by: dividing O by it makes O an exact convex
-                            // combination of V rows (a lone dominant weight is not rounded away)
+        RowState st;  // lr: dividing O by it makes O an exact convex combination of V rows
+                      // (a lone dominant weight is not rounded away)
         for (int j = 0; j < n; ++j, ++gs) {
             ok = mbar_wait(s_full, gs & 1, abort_flag, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
 
-            const int kv0 = (u.lo + j) * BN;
-            const bool masked = kv0 + BN > lim;  // masking step: keys at or beyond the row's limit
             float s[BN];
             uint32_t pk0[32], pk1[32];          // P for keys [0,64) and [64,128), two bf16 per column
             float2 ls = make_float2(0.f, 0.f);  // this tile's unrounded sum (packed pair)
-            float lrs = 0.f;                    // this tile's rounded (bf16) sum
-            // the row's 128 scores: four 32-column TMEM loads, one wait
-            tmem_ld32f(t_s + 0, s);
-            tmem_ld32f(t_s + 32, s + 32);
-            tmem_ld32f(t_s + 64, s + 64);
-            tmem_ld32f(t_s + 96, s + 96);
-            tmem_ld_wait();
-            tmem_reg_fence_f<BN>(s);
-            if (masked) {
-                mask_scores<0>(s, kv0, lim);
-                mask_scores<1>(s, kv0, lim);
+            load_score_row(t_s, s);
+            if constexpr (kSep) {  // S_X is in registers: its columns may take the next Q_X K^T
+                tc_fence_before();
+                mbar_arrive(s_free);
             }
-            const float m_new = fmaxf(max64(s), max64(s + 64)) * p.scale_log2;
-            float alpha = 1.f;
-            bool resc = false;
-            if (j == 0) {
-                m_ref = (m_new == NEG_INF) ? 0.f : m_new;
-                l = 0.f;
-                lr = 0.f;
-            } else if (m_new > m_ref + p.tau) {
-                alpha = ex2_approx(m_ref - m_new);
-                l *= alpha;
-                lr *= alpha;
-                m_ref = m_new;
-                resc = true;
-            }
+            const float m_new = masked_row_max(s, (u.lo + j) * BN, lim, p.scale_log2);
+            float alpha;
+            const bool resc = update_reference(st, j, m_new, p.tau, alpha);
             if (__any_sync(0xffffffffu, resc)) {
                 // O_X holds P_X V for key tiles < j and nothing is adding to it:
-                // the commit that released S_X(j) covered the last such product,
-                // and the next one waits for this tile's P.  Scale in place.
-#pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
-                    uint32_t r[32];
-                    tmem_ld32(t_o + ch * 32, r);
-                    tmem_ld_wait();
-                    tmem_reg_fence(r);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-                    tmem_st32(t_o + ch * 32, r);
+                // the commit that released S_X(j) covered the last such product
+                // (separate P: the wait below does), and the next one waits for
+                // this tile's P.  Scale in place.
+                if constexpr (kSep) {
+                    if (!(ok = ensure_pv(gs))) break;
+                    tc_fence_after();
                 }
+                rescale_o_row<D>(t_o, alpha);
             }
             if constexpr (F8) {
-                exp_e4m3(s, p.scale_log2, kF8Shift - m_ref, pk0, ls);
+                exp_e4m3(s, p.scale_log2, kF8Shift - st.m_ref, pk0, ls);
                 tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
-            } else if constexpr (kLateSums) {
-                exp_half_p<0>(s, p.scale_log2, -m_ref, pk0, ls);
-                tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
-                if constexpr (kSplitPV<D>) {
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(p_half);
-                }
-                exp_half_p<1>(s, p.scale_log2, -m_ref, pk1, ls);
-                tmem_st32(t_s + 32, pk1);
+            } else if constexpr (kSep) {
+                exp_half_p<0>(s, p.scale_log2, -st.m_ref, pk0, ls);
+                exp_half_p<1>(s, p.scale_log2, -st.m_ref, pk1, ls);
+                // P_X(j - 1) must have been read by its product before it is replaced
+                if (!(ok = ensure_pv(gs))) break;
+                tc_fence_after();
+                tmem_st32(t_p + 0, pk0);
+                tmem_st32(t_p + 32, pk1);
             } else {
-                exp_half<0>(s, p.scale_log2, -m_ref, pk0, ls, lrs);
+                exp_half_p<0>(s, p.scale_log2, -st.m_ref, pk0, ls);
                 tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
-                if constexpr (kSplitPV<D>) {
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(p_half);
-                }
-                exp_half<1>(s, p.scale_log2, -m_ref, pk1, ls, lrs);
+                exp_half_p<1>(s, p.scale_log2, -st.m_ref, pk1, ls);
                 tmem_st32(t_s + 32, pk1);
             }
-            if constexpr (!F8 && kLateSums) {
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(p_full);
-                l += ls.x + ls.y;
-                lr += rounded_sum(pk0, pk1);
-            } else {
-                l += ls.x + ls.y;
-                lr += lrs;
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(p_full);
-            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(p_full);
+            // the sums after the "P ready" signal, so that the tensor core gets P
+            // sooner: the unrounded one (lse) and, bf16 only, the sum of the
+            // rounded probabilities from the packed pairs still in registers
+            st.l += ls.x + ls.y;
+            if constexpr (!F8) st.lr += rounded_sum(pk0, pk1);
         }
         if (ok) {
-            ok = mbar_wait(o_final, tl & 1, abort_flag, p.timeout_ns);
-            ok = __all_sync(0xffffffffu, ok);
+            if constexpr (kSep) {
+                ok = ensure_pv(gs);  // every product of this unit
+            } else {
+                ok = mbar_wait(o_final, tl & 1, abort_flag, p.timeout_ns);
+                ok = __all_sync(0xffffffffu, ok);
+            }
         }
         if (!ok) {  // abandon this unit: mark its rows
             if (row_valid) fill_row<D, O_BF16>(p.o, p.lse, row_id, true, __int_as_float(0x7fc00000));
@@ -602,22 +483,20 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         }
         tc_fence_after();
         // a row whose allowed keys all lie outside this unit's key range (key
-        // splits) has nothing summed: O = 0, lse = -inf for it
-        // E4M3: O over the unrounded sum (with eager rescaling the row maximum's
-        // weight 2^8 is exact in E4M3, so the rounded and unrounded sums differ
-        // only by the unbiased rounding of the smaller weights)
-        const float norm = F8 ? l : lr;
-        const bool empty = !(norm > 0.f);
-        const float inv_l = empty ? 0.f : (F8 ? p.out_scale : 1.f) / norm;
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t r[32];
-            tmem_ld32(t_o + ch * 32, r);
-            tmem_ld_wait();
-            tmem_reg_fence(r);
-            if (row_valid) store_row_chunk<D, O_BF16>(p.o, row_id, ch, r, inv_l);
+        // splits) has nothing summed: O = 0, lse = -inf for it.  E4M3: O over
+        // the unrounded sum (with eager rescaling the row maximum's weight 2^8
+        // is exact in E4M3, so the rounded and unrounded sums differ only by
+        // the unbiased rounding of the smaller weights)
+        if constexpr (C::kStageO && !O_BF16) {
+            // the warp's 32 rows are consecutive output rows starting at lane 0's
+            const size_t first_row_id = row_id - lane;
+            const int n_valid = min(32, p.N - (row - lane));
+            write_rows_coalesced<D>(t_o, stage, lane, static_cast<float *>(p.o), p.lse, first_row_id, n_valid, st.lr,
+                                    st.m_ref + log2f(st.l));
+        } else {
+            write_row<D, O_BF16>(t_o, p.o, p.lse, row_id, row_valid, F8 ? st.l : st.lr, F8 ? p.out_scale : 1.f,
+                                 st.m_ref - (F8 ? kF8Shift : 0.f) + log2f(st.l));
         }
-        if (row_valid) p.lse[row_id] = empty ? NEG_INF : (m_ref - (F8 ? kF8Shift : 0.f) + log2f(l)) * LN2;
         tc_fence_before();
         mbar_arrive(o_free);
         ++tl;
@@ -663,16 +542,6 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
             if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
             tc_fence_after();
             mma_e4m3_ts_k128(tmem + col_o(x, D), tmem + col_s(x), vd, idesc_pv, first ? 0u : 1u);
-        } else if constexpr (kSplitPV<D>) {
-            // keys [0, 64): P columns [0, 32), V rows [0, 64); then keys [64, 128)
-            if (!mbar_wait(&bars[C::kBarPHalf + x], gpx & 1, abort_flag, to)) return false;
-            if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
-            tc_fence_after();
-            mma_ts_k64(tmem + col_o(x, D), tmem + col_s(x), vd, idesc_pv, first ? 0u : 1u);
-            if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
-            ++gpx;
-            tc_fence_after();
-            mma_ts_k64(tmem + col_o(x, D), tmem + col_s(x) + 32, vd + (4 * 2048 >> 4), idesc_pv, 1u);
         } else {
             if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
             ++gpx;
@@ -684,18 +553,66 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
         return true;
     };
 
+    // separate P (d = 64): per key tile j, Q_A K_j^T and Q_B K_j^T as soon as
+    // the softmax has read S_X(j - 1), then P_A V_{j-1} and P_B V_{j-1}
+    uint32_t gq0 = 0, gq1 = 0;    // Q_X K^T products issued (s_free phase)
+    auto qk_sep = [&](int x, uint32_t &gqx, uint32_t kslot) -> bool {
+        if (gqx > 0 && !mbar_wait(&bars[C::kBarSFree + x], (gqx - 1) & 1, abort_flag, to)) return false;
+        ++gqx;
+        tc_fence_after();
+        qk(x, kslot);
+        return true;
+    };
+    auto pv_sep = [&](int x, uint32_t &gpx, uint32_t tlx, uint32_t vslot, bool first) -> bool {
+        if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
+        ++gpx;
+        if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
+        tc_fence_after();
+        mma_ts_k128(tmem + col_o(x, D), tmem + col_p_sep(x), v_desc + ((vslot * C::kTileBytes) >> 4), idesc_pv,
+                    first ? 0u : 1u);
+        tc_commit(&bars[C::kBarPvDone + x]);
+        return true;
+    };
+
     bool ok = true;
     for (int k = 0; ok; ++k) {
         UnitCoord u;  // dynamic: the key-tile counts come with the id (the TMA warp decoded the unit)
         const int t = p.dynamic ? unit_pop(uq, k, abort_flag, to, ok, &u.n[0], &u.n[1]) : unit_static(p, k);
         if (!ok || t < 0) break;
-        if (!p.dynamic) u = decode_unit(p, t);
+        if (!p.dynamic) u = decode_unit(p, t, uq.b_order);
         u.nmax = max(u.n[0], u.n[1]);
         if (u.nmax == 0) continue;
         if (!mbar_wait(&bars[C::kBarQFull], tq & 1, abort_flag, to)) { ok = false; break; }
         ++tq;
         tc_fence_after();
-        for (int j = 0; j <= u.nmax; ++j) {
+        if constexpr (kSepP<D> && !F8) {
+            for (int j = 0; j <= u.nmax && ok; ++j) {
+                if (j < u.nmax) {
+                    const uint32_t kslot = gk % C::kKStages;
+                    if (!mbar_wait(&bars[C::kBarKFull + kslot], (gk / C::kKStages) & 1, abort_flag, to)) {
+                        ok = false;
+                        break;
+                    }
+                    if (j < u.n[0] && !qk_sep(0, gq0, kslot)) { ok = false; break; }
+                    if (j < u.n[1] && !qk_sep(1, gq1, kslot)) { ok = false; break; }
+                    tc_commit(&bars[C::kBarKEmpty + kslot]);
+                    ++gk;
+                    if (j == u.nmax - 1) tc_commit(&bars[C::kBarQEmpty]);
+                }
+                if (j > 0) {
+                    const uint32_t vslot = gv % C::kVStages;
+                    if (!mbar_wait(&bars[C::kBarVFull + vslot], (gv / C::kVStages) & 1, abort_flag, to)) {
+                        ok = false;
+                        break;
+                    }
+                    if (j - 1 < u.n[0] && !pv_sep(0, gp0, tl0, vslot, j == 1)) { ok = false; break; }
+                    if (j - 1 < u.n[1] && !pv_sep(1, gp1, tl1, vslot, j == 1)) { ok = false; break; }
+                    tc_commit(&bars[C::kBarVEmpty + vslot]);
+                    ++gv;
+                }
+            }
+        } else {
+          for (int j = 0; j <= u.nmax; ++j) {
             // products with V_{j-1}, interleaved with the scores of key tile j
             const bool have_k = j < u.nmax;
             const uint32_t kslot = gk % C::kKStages, vslot = gv % C::kVStages;
@@ -725,6 +642,7 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
                 ++gk;
                 if (j == u.nmax - 1) tc_commit(&bars[C::kBarQEmpty]);
             }
+          }
         }
         tl0 += u.n[0] > 0;
         tl1 += u.n[1] > 0;
@@ -742,6 +660,8 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
     prefetch_tensormap(&p.tm_v);
     const uint64_t to = p.timeout_ns;
     uint32_t tq = 0, gk = 0, gv = 0;
+    // test only: the K load this CTA never issues (its ring position), or none
+    const uint32_t drop = (blockIdx.x == 0 && p.drop_load > 0) ? (uint32_t)(p.drop_load - 1) : 0xFFFFFFFFu;
     bool ok = true;
     for (int k = 0; ok; ++k) {
         const int t = p.dynamic ? unit_take(p, uq, k, abort_flag, to, ok) : unit_static(p, k);
@@ -750,7 +670,7 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
             if (p.dynamic) unit_publish(uq, k, -1, 0, 0);
             break;
         }
-        const UnitCoord u = decode_unit(p, t);
+        const UnitCoord u = decode_unit(p, t, uq.b_order);
         if (p.dynamic) unit_publish(uq, k, t, u.n[0], u.n[1]);
         if (u.nmax == 0) continue;
         if (tq > 0 && !mbar_wait(&bars[C::kBarQEmpty], (tq - 1) & 1, abort_flag, to)) {
@@ -772,11 +692,13 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&bars[C::kBarKFull + slot], C::kTileBytes);
+                if (gk != drop) {
+                    mbar_arrive_expect_tx(&bars[C::kBarKFull + slot], C::kTileBytes);
 #pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(sK + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_k, &bars[C::kBarKFull + slot],
-                                c * C::kChunkElems, (u.lo + j) * BN, u.bh_kv);
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(sK + slot * C::kTileBytes + c * C::kChunkBytes, &p.tm_k,
+                                    &bars[C::kBarKFull + slot], c * C::kChunkElems, (u.lo + j) * BN, u.bh_kv);
+                }
                 ++gk;
             }
             {
@@ -796,16 +718,16 @@ __device__ __forceinline__ void load_role(const FwdParams &p, uint64_t *bars, vo
     }
     if (!ok) record_timeout(p);
     // drain: every copy this thread issued has landed before the CTA may exit
-    if (tq > 0) mbar_wait_drain(&bars[C::kBarQFull], (tq - 1) & 1, to);
+    if (tq > 0) mbar_wait_drain(&bars[C::kBarQFull], (tq - 1) & 1);
     const uint32_t nk = gk < (uint32_t)C::kKStages ? gk : (uint32_t)C::kKStages;
     for (uint32_t i = 0; i < nk; ++i) {
         const uint32_t g = gk - 1 - i;
-        mbar_wait_drain(&bars[C::kBarKFull + g % C::kKStages], (g / C::kKStages) & 1, to);
+        if (g != drop) mbar_wait_drain(&bars[C::kBarKFull + g % C::kKStages], (g / C::kKStages) & 1);
     }
     const uint32_t nv = gv < (uint32_t)C::kVStages ? gv : (uint32_t)C::kVStages;
     for (uint32_t i = 0; i < nv; ++i) {
         const uint32_t g = gv - 1 - i;
-        mbar_wait_drain(&bars[C::kBarVFull + g % C::kVStages], (g / C::kVStages) & 1, to);
+        mbar_wait_drain(&bars[C::kBarVFull + g % C::kVStages], (g / C::kVStages) & 1);
     }
 }
 
@@ -825,18 +747,40 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    int *b_order = reinterpret_cast<int *>(smem + C::kOffBOrder);
     const UnitQueue uq{reinterpret_cast<volatile int *>(smem + C::kOffUnitIds), &bars[C::kBarUnitFull],
-                       &bars[C::kBarUnitFree]};
+                       &bars[C::kBarUnitFree], p.sort_b ? b_order : nullptr};
+    if (p.sort_b) {
+        // rank of batch element t among all by (key tiles descending, index):
+        // its key tiles first go to the table, then every thread t < B counts
+        // the elements ahead of it and writes t at its rank
+        const int t = threadIdx.x;
+        int tiles = 0, rank = 0;
+        if (t < p.B) {
+            tiles = (min(max(__ldg(p.k_len + t), 0), p.Nk) + BN - 1) / BN;
+            b_order[t] = tiles;
+        }
+        __syncthreads();
+        if (t < p.B)
+            for (int i = 0; i < p.B; ++i) {
+                const int ti = b_order[i];
+                rank += (ti > tiles) || (ti == tiles && i < t);
+            }
+        __syncthreads();
+        if (t < p.B) b_order[rank] = t;
+    }
+    volatile int *claimed = reinterpret_cast<volatile int *>(smem + C::kOffClaimed);
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
             const bool per_row = (i >= C::kBarPFull && i < C::kBarPFull + 2) ||
                                  (i >= C::kBarOFree && i < C::kBarOFree + 2) ||
-                                 (i >= C::kBarPHalf && i < C::kBarPHalf + 2);
+                                 (i >= C::kBarSFree && i < C::kBarSFree + 2);
             // a queued unit id is read by the 256 softmax threads and the MMA thread
             const bool unit_free = i >= C::kBarUnitFree && i < C::kBarUnitFree + kUnitQueue;
             mbar_init(&bars[i], unit_free ? 2u * 128u + 1u : (per_row ? 128u : 1u));
         }
         *abort_flag = 0;
+        *claimed = p.dynamic ? (sched_claim(p.sched, p.timeout_ns) ? 1 : 0) : 1;
         fence_mbar_init();
     }
     if (warp == kMmaWarp) {
@@ -847,10 +791,17 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (!*claimed) {  // the scheduler slot stayed in use by another launch: no work, report it
+        if (threadIdx.x == 0) record_status(p.status, kStatusSchedBusy);
+        if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+        return;
+    }
 
     if (warp < kSoftmaxWarps) {
         setmaxnreg_inc<kSoftmaxRegs>();
-        if (!softmax_role<D, O_BF16, F8>(p, bars, abort_flag, uq, tmem, warp >> 2, warp, lane)) record_timeout(p);
+        float *stage = reinterpret_cast<float *>(smem + C::kOffStage) + warp * 32 * 36;
+        if (!softmax_role<D, O_BF16, F8>(p, bars, abort_flag, uq, tmem, warp >> 2, warp, lane, stage))
+            record_timeout(p);
     } else {
         setmaxnreg_dec<kControlRegs>();
     }
@@ -860,7 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
                 record_timeout(p);
             // drain: no MMA may still be running when TMEM is released
             tc_commit(&bars[C::kBarDrain]);
-            mbar_wait_drain(&bars[C::kBarDrain], 0, p.timeout_ns);
+            mbar_wait_drain(&bars[C::kBarDrain], 0);
         }
     } else if (warp == kLoadWarp) {
         if (lane == 0) load_role<D, F8>(p, bars, abort_flag, uq, sQ, sK, sV);

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_internal.h"
 
 namespace {
 
@@ -50,16 +51,20 @@ fa_status scratch_for_current_device(void **out) {
 extern "C" {
 
 fa_status fa_fwd_static_workspace(const fa_fwd_params *p, void *stream) {
-    if (!p) return FA_ERR_INVALID_ARGUMENT;
+    // order: argument checks (no CUDA call), the size limit, the device, then
+    // the array's address
+    fa_status st = fa_detail::validate_args(p);
+    if (st != FA_OK) return st;
+    if ((long long)p->B * p->H * p->N == 0) return FA_OK;
     fa_fwd_params c = *p;
     c.workspace = nullptr;
     c.workspace_bytes = 0;
     if (c.num_splits > 1) {
         const size_t need = fa_fwd_workspace_bytes(&c);
         if (need > (size_t)FA_STATIC_WORKSPACE_BYTES) return FA_ERR_WORKSPACE_LIMIT;
+        if ((st = fa_detail::probe_current_device()) != FA_OK) return st;
         void *ws = nullptr;
-        const fa_status st = scratch_for_current_device(&ws);
-        if (st != FA_OK) return st;
+        if ((st = scratch_for_current_device(&ws)) != FA_OK) return st;
         c.workspace = ws;
         c.workspace_bytes = (size_t)FA_STATIC_WORKSPACE_BYTES;
     }

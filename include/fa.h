@@ -62,8 +62,11 @@ typedef enum {
     FA_ERR_UNSUPPORTED = 3,      /* d not in {64, 128, 256}, or the device is not sm_100 */
     FA_ERR_CUDA = 4,             /* a CUDA runtime/driver call or the launch failed   */
     FA_ERR_DEVICE_TIMEOUT = 5,   /* (device status word) a pipeline wait timed out     */
-    FA_ERR_WORKSPACE_LIMIT = 6   /* fa_fwd_static_workspace: the splits need more than
+    FA_ERR_WORKSPACE_LIMIT = 6,  /* fa_fwd_static_workspace: the splits need more than
                                     FA_STATIC_WORKSPACE_BYTES of scratch                */
+    FA_ERR_SCHED_BUSY = 7        /* (device status word) the launch's scheduler slot stayed
+                                    in use by another in-flight launch for longer than the
+                                    wait limit; the launch did no work                  */
 } fa_status;
 
 typedef enum { FA_O_F32 = 0, FA_O_BF16 = 1 } fa_o_dtype;
@@ -134,6 +137,12 @@ typedef struct {
                                 for bf16.  The products Q K^T and P V run on E4M3 with
                                 fp32 accumulation; P is rounded to E4M3 before P V;
                                 the softmax is fp32.  Finite and >= 0.                */
+    int test_drop_load;      /* test only; 0 (off) in every normal call.  n > 0: the TMA
+                                producer of the kernel's first CTA never issues its n-th
+                                key-tile load (d = 256: its n-th K/V half-tile load), so
+                                the pipeline wait for that tile runs out after timeout_ms
+                                and the time-out path (status word, NaN rows, drain,
+                                exit) runs with no copy in flight.  Must be >= 0.       */
 } fa_fwd_params;
 
 /*
@@ -156,11 +165,27 @@ FA_EXPORT int fa_fwd_suggest_splits(const fa_fwd_params *p);
 /*
  * fa_fwd_ex -- the forward pass with key padding, output dtype and a status
  * word.  Causal problems hand their work units out through a per-launch
- * counter held by the library (64 slots per device, taken round-robin): at
- * most 64 causal fa_fwd / fa_fwd_ex / fa_bwd launches may be in flight on one
- * device at the same time, on any streams.  On a device-side timeout the kernel stores FA_ERR_DEVICE_TIMEOUT in
- * *dev_status, stops, writes NaN to the rows of the tile it was working on
- * and leaves the rows of unprocessed tiles unwritten.
+ * counter held by the library (64 slots per device, taken round-robin by
+ * causal fa_fwd / fa_fwd_ex / fa_bwd launches).  Each launch's CTAs claim its
+ * slot for their grid before taking a unit, so launches that meet on a slot
+ * (more than 64 in flight at once on one device, or one CUDA graph replayed
+ * on several streams) run one after the other instead of sharing a counter;
+ * a launch whose wait for its slot outlasts timeout_ms does no work and
+ * stores FA_ERR_SCHED_BUSY in *dev_status.
+ *
+ * On a device-side timeout the kernel stores FA_ERR_DEVICE_TIMEOUT in
+ * *dev_status and stops: the CTA that timed out writes NaN to the rows of the
+ * unit it was working on, but its remaining units are never written, and
+ * with key splits the merge still runs over whatever partials the workspace
+ * holds.  After FA_ERR_DEVICE_TIMEOUT the whole of o and lse is undefined;
+ * the error is seen only through the status word, so pass one when the
+ * result matters.
+ *
+ * The library caches device addresses (its scheduler words, and the scratch
+ * array of fa_fwd_static_workspace) per device ordinal for the life of the
+ * process.  Do not reset a device (cudaDeviceReset) between calls into this
+ * library: the module is reloaded at a possibly different address and the
+ * cached addresses would be stale.
  */
 FA_EXPORT fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream);
 
@@ -266,6 +291,19 @@ FA_EXPORT fa_status fa_bwd(const fa_bwd_params *p, void *stream);
  * FA_ERR_WORKSPACE_LIMIT, and FA_ERR_CUDA if the lookup fails.
  */
 FA_EXPORT fa_status fa_fwd_static_workspace(const fa_fwd_params *p, void *stream);
+
+/*
+ * Test hooks (not for production use): the scheduler slot the next causal
+ * launch from this process will take, and a synchronous read (get4) and/or
+ * overwrite (set4) of a slot's four words on the current device ([0] next
+ * unit, [1] CTAs done, [2..3] the 64-bit owner, little-endian; all zero when
+ * the slot is free).  They let a test hold a slot the way an in-flight
+ * launch would, without a second launch.  Errors: FA_ERR_INVALID_ARGUMENT
+ * for a slot outside [0, 64), FA_ERR_UNSUPPORTED / FA_ERR_CUDA from the
+ * device.
+ */
+FA_EXPORT int fa_testhook_sched_next_slot(void);
+FA_EXPORT fa_status fa_testhook_sched_slot(int slot, const uint32_t *set4, uint32_t *get4);
 
 #ifdef __cplusplus
 }

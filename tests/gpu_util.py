@@ -15,29 +15,65 @@ TOL_MEAN = 1e-3   # mean |O_gpu - O_ref|
 TOL_LSE = 1e-4    # max |lse_gpu - lse_ref| / max(|lse_ref|, 1)
 
 
+# Guard regions: every output buffer a GPU test hands to the library sits
+# between two runs of GUARD_BYTES bytes of a fixed pattern, checked bit for bit
+# after the call, so a store past either end of a buffer (a wrong row index, a
+# ragged tail, a split layout off by one) fails the test instead of silently
+# corrupting a neighbour.
+GUARD_BYTES = 4096
+GUARD_BYTE = 0xA5
+
+
+class Guarded:
+    """A device tensor of `shape` and `dtype` with guard bytes on both sides."""
+
+    def __init__(self, shape, dtype, dev, fill=None):
+        esize = torch.empty((), dtype=dtype).element_size()
+        self.nbytes = int(np.prod(shape)) * esize
+        self.buf = torch.full((2 * GUARD_BYTES + self.nbytes,), GUARD_BYTE, dtype=torch.uint8, device=dev)
+        self.t = self.buf[GUARD_BYTES:GUARD_BYTES + self.nbytes].view(dtype).view(shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def check(self, name="buffer"):
+        head = self.buf[:GUARD_BYTES]
+        tail = self.buf[GUARD_BYTES + self.nbytes:]
+        bad_head = int((head != GUARD_BYTE).sum())
+        bad_tail = int((tail != GUARD_BYTE).sum())
+        assert bad_head == 0 and bad_tail == 0, \
+            f"{name}: {bad_head} guard bytes changed before and {bad_tail} after the buffer"
+
+
 def run_gpu(q, k, v, causal, scale, k_len=None, out_dtype=torch.float32, flags=0, stream=None, num_splits=0,
             descale=(0.0, 0.0, 0.0)):
     """Run fa_fwd_ex on cuda:0; returns (O [B,H,N,d] fp32 CPU, lse [B,H,N] CPU).
 
     Outputs (and any split workspace) start as NaN so rows the kernels fail to
-    write are caught.  num_splits = -1 takes the library's suggestion."""
+    write are caught, and sit between guard regions that must come back
+    untouched.  num_splits = -1 takes the library's suggestion."""
     dev = torch.device("cuda:0")
     B, H, N, d = q.shape
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
     kl = None if k_len is None else torch.as_tensor(k_len, dtype=torch.int32).to(dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    o = torch.full((B, H, N, d), float("nan"), dtype=out_dtype, device=dev)
-    lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
+    og = Guarded((B, H, N, d), out_dtype, dev, fill=float("nan"))
+    lg = Guarded((B, H, N), torch.float32, dev, fill=float("nan"))
+    o, lse = og.t, lg.t
     if num_splits < 0:
         num_splits = fb.suggest_splits(qd, kd)
-    ws = None
+    wg, ws = None, None
     if num_splits > 1:
         nbytes = fb.workspace_bytes(qd, kd, num_splits)
-        ws = torch.full((max(nbytes, 16) // 4,), float("nan"), dtype=torch.float32, device=dev)
+        wg = Guarded((max(nbytes, 16) // 4,), torch.float32, dev, fill=float("nan"))
+        ws = wg.t
     fb.fa_fwd_ex(qd, kd, vd, o, lse, causal, scale, k_len=kl, dev_status=status, flags=flags, stream=stream,
                  num_splits=num_splits, workspace=ws, descale=descale)
     st = fb.read_device_status(status, stream=stream)
     assert st == fb.FA_OK, fb.status_string(st)
+    og.check("o")
+    lg.check("lse")
+    if wg is not None:
+        wg.check("workspace")
     return o.float().cpu(), lse.cpu()
 
 

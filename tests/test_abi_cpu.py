@@ -145,6 +145,14 @@ def test_static_workspace_entry_validates():
     assert lib.fa_fwd_static_workspace(ctypes.byref(_params(d=32)), None) == fb.FA_ERR_UNSUPPORTED
     assert lib.fa_fwd_static_workspace(ctypes.byref(_params(q=None)), None) == fb.FA_ERR_INVALID_ARGUMENT
     assert lib.fa_fwd_static_workspace(ctypes.byref(_params(N=0)), None) == fb.FA_OK
+    # with splits, the argument checks still come first and make no CUDA call
+    # (on a host without a GPU a CUDA call would turn these into FA_ERR_CUDA)
+    assert lib.fa_fwd_static_workspace(ctypes.byref(_params(q=None, num_splits=4)), None) == \
+        fb.FA_ERR_INVALID_ARGUMENT
+    assert lib.fa_fwd_static_workspace(ctypes.byref(_params(num_splits=2000)), None) == fb.FA_ERR_INVALID_ARGUMENT
+    assert lib.fa_fwd_static_workspace(ctypes.byref(_params(o=0x40008, num_splits=4)), None) == \
+        fb.FA_ERR_MISALIGNED
+    assert lib.fa_fwd_static_workspace(ctypes.byref(_params(d=32, num_splits=4)), None) == fb.FA_ERR_UNSUPPORTED
 
 
 def test_host_entry_validates():

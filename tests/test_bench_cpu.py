@@ -126,3 +126,56 @@ def test_committed_records_name_existing_sources():
             assert os.path.isfile(os.path.join(bench.ROOT, "exact_io_aware_52_b200", "csrc", name)), (path, name)
         assert len(rec["source_hash"]) == 16 and int(rec["source_hash"], 16) >= 0
         assert float(rec["dram_bytes_per_launch"]) == float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])
+
+
+def test_clock_peak_is_sms_times_8192_per_clock():
+    # 148 SMs at 1965 MHz: 148 * 8192 * 1.965e9 = 2382.4 TFLOP/s
+    assert abs(bench.clock_peak_tflops(148, 1965.0) - 148 * 8192 * 1.965e9 / 1e12) < 1e-9
+    assert abs(bench.clock_peak_tflops(148, 1000.0, ratio=2.0) - 2 * 148 * 8192 * 1e9 / 1e12) < 1e-9
+
+
+def test_percentiles_match_numpy_linear_interpolation():
+    rng = np.random.default_rng(3)
+    xs = rng.exponential(size=37).tolist()
+    st = bench.percentiles(xs)
+    for key, q in (("median", 50), ("p10", 10), ("p90", 90)):
+        assert abs(st[key] - float(np.percentile(xs, q))) < 1e-12
+    assert abs(st["mean"] - float(np.mean(xs))) < 1e-12 and st["n"] == 37
+    assert bench.percentiles([2.5]) == {"median": 2.5, "p10": 2.5, "p90": 2.5, "mean": 2.5, "n": 1}
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_effective_flops_count_keys_inside_each_length(causal):
+    w = workloads.custom(3, 2, 40, 64, causal=causal, Nk=56)
+    k_len = [56, 0, 23]
+    expect = sum(4.0 * 2 * 64 * _allowed_pairs(40, 56, causal, k_len=L) for L in k_len)
+    assert bench.effective_flops(w, k_len) == expect
+    assert bench.effective_flops(w, None) == w.flops()
+
+
+def test_bert_shaped_effective_flops_follow_the_drawn_lengths():
+    w = workloads.WORKLOADS[3]
+    _, _, _, k_len = workloads.make_inputs(w)
+    L = k_len.tolist()
+    assert all(256 <= x <= 512 for x in L)
+    assert bench.effective_flops(w, L) == 4.0 * w.H * w.N * w.d * sum(L)
+    assert bench.effective_flops(w, L) < w.flops()
+
+
+def test_guard_regions_catch_writes_past_either_end():
+    """The guard helper the GPU tests wrap every output buffer in, exercised on
+    CPU tensors: untouched guards pass; one byte changed on either side fails."""
+    import torch
+
+    from tests.gpu_util import GUARD_BYTES, Guarded
+    g = Guarded((3, 5), torch.float32, "cpu", fill=float("nan"))
+    assert g.t.shape == (3, 5) and bool(torch.isnan(g.t).all())
+    g.t.fill_(1.0)
+    g.check("ok")
+    g.buf[GUARD_BYTES + g.nbytes] = 0  # one byte past the end
+    with pytest.raises(AssertionError, match="after"):
+        g.check("tail")
+    g2 = Guarded((7,), torch.float32, "cpu")
+    g2.buf[GUARD_BYTES - 1] = 1  # one byte before the start
+    with pytest.raises(AssertionError, match="1 guard bytes changed before"):
+        g2.check("head")

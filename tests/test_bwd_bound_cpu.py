@@ -45,3 +45,18 @@ def test_bound_holds_for_the_rounding_model():
             err = np.abs(emul - ref)
             assert np.all(err <= bnd), name
             assert err.max() > 0.02 * bnd.max(), name  # not vacuously loose
+
+
+def test_row_chunks_give_the_same_bound():
+    """Taking the query rows in chunks changes nothing but the order of the dK
+    and dV bound sums (every other quantity of a row depends on that row)."""
+    g = torch.Generator().manual_seed(10)
+    B, H, H_kv, N, Nk, d = 2, 2, 1, 37, 50, 16
+    q, do = (torch.randn(B, H, N, d, generator=g).double().numpy() for _ in range(2))
+    k, v = (torch.randn(B, H_kv, Nk, d, generator=g).double().numpy() for _ in range(2))
+    for causal in (False, True):
+        whole = bwd_bound.bounds(q, k, v, do, causal, 0.25, k_len=[50, 20], row_chunk=N)
+        for chunk in (1, 5, 16):
+            part = bwd_bound.bounds(q, k, v, do, causal, 0.25, k_len=[50, 20], row_chunk=chunk)
+            for a, b in zip(whole, part):
+                np.testing.assert_allclose(a, b, rtol=1e-12, atol=0)

@@ -15,7 +15,7 @@ import oracle
 from exact_io_aware_52_b200 import _binding as fb
 from exact_io_aware_52_b200 import workloads
 from tests import bwd_bound
-from tests.gpu_util import run_gpu
+from tests.gpu_util import Guarded, run_gpu
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -36,13 +36,17 @@ def run_bwd(q, k, v, do, o, lse, causal, scale, k_len=None):
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
     qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
     od, lsed = o.to(DEV), lse.to(DEV)
-    dq = torch.full(q.shape, float("nan"), device=DEV)
-    dk = torch.full(k.shape, float("nan"), device=DEV)
-    dv = torch.full(v.shape, float("nan"), device=DEV)
-    ws = torch.empty(max(fb.bwd_workspace_bytes(q), 16), dtype=torch.uint8, device=DEV)
+    # gradients and the D workspace between guard regions (tests.gpu_util.Guarded)
+    gq = Guarded(tuple(q.shape), torch.float32, DEV, fill=float("nan"))
+    gk = Guarded(tuple(k.shape), torch.float32, DEV, fill=float("nan"))
+    gv = Guarded(tuple(v.shape), torch.float32, DEV, fill=float("nan"))
+    gw = Guarded((max(fb.bwd_workspace_bytes(q), 16),), torch.uint8, DEV)
+    dq, dk, dv, ws = gq.t, gk.t, gv.t, gw.t
     kl = None if k_len is None else torch.tensor(k_len, dtype=torch.int32, device=DEV)
     fb.fa_bwd(qd, kd, vd, od, lsed, dod, dq, dk, dv, causal, scale, ws, k_len=kl, dev_status=st)
     assert fb.read_device_status(st) == fb.FA_OK
+    for g, name in ((gq, "dq"), (gk, "dk"), (gv, "dv"), (gw, "workspace")):
+        g.check(name)
     return dq.cpu().double().numpy(), dk.cpu().double().numpy(), dv.cpu().double().numpy()
 
 
@@ -129,6 +133,34 @@ def test_full_size_invariants():
     assert np.all(np.abs(dk.sum(2)) <= 1e-3 * col + 1e-3)
     dsum = do.double().numpy().sum(2)
     assert np.all(np.abs(dv.sum(2) - dsum) <= 1e-3 * np.abs(do.double().numpy()).sum(2) + 1e-3)
+
+
+def test_full_size_two_heads_element_wise():
+    """The full long-context shape (B1 H32 N16384 d128 causal, the backward
+    benchmark's launch configuration: banded unit order, 128-tile query loops),
+    compared element by element with the fp64 backward oracle on two of its
+    heads under the derived bound.  Heads are independent in the definition,
+    so the oracle runs on those heads alone; their O and lse are the forward
+    oracle's (the other heads keep the forward kernel's, which cannot reach
+    the checked heads' gradients)."""
+    w = workloads.WORKLOADS[10]
+    q, k, v, _ = workloads.make_inputs(w)
+    do = workloads.make_dout(w)
+    heads = [0, w.H - 1]
+    sub = [t[:, heads].contiguous() for t in (q, k, v, do)]
+    o, lse = run_gpu(q, k, v, True, w.scale)
+    o_ref, lse_ref = oracle.attention_f64(sub[0], sub[1], sub[2], True, w.scale)
+    o[:, heads] = torch.from_numpy(o_ref.reshape(1, 2, w.N, w.d)).float()
+    lse[:, heads] = torch.from_numpy(lse_ref.reshape(1, 2, w.N)).float()
+    got = run_bwd(q, k, v, do, o, lse, True, w.scale)
+    ref = oracle.attention_bwd_f64(*sub, True, w.scale, nthreads=2)
+    bnd = bwd_bound.bounds(*(t.double().numpy() for t in sub), True, float(np.float32(w.scale)))
+    for name, a, b, c in zip(("dq", "dk", "dv"), got, ref, bnd):
+        a = a[:, heads]
+        assert np.all(np.isfinite(a)), name
+        err = np.abs(a - b)
+        worst = np.unravel_index(np.argmax(err / c), err.shape)
+        assert np.all(err <= c), (name, float(err[worst]), float(c[worst]), worst)
 
 
 def test_deterministic_dk_dv():

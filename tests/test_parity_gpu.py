@@ -63,6 +63,20 @@ def test_key_padding_edges(d, causal):
     check_case(q, k, v, causal, 1.0 / math.sqrt(d), k_len=k_len)
 
 
+@pytest.mark.parametrize("B", [127, 128, 129])
+def test_key_padding_many_batch_elements(B):
+    """Key-padded non-causal problems hand their units out longest batch
+    element first (an order table of up to 128 elements built in each CTA);
+    beyond 128 elements they keep the static order.  Both sides of that
+    limit, with lengths that tie, differ and are empty, against the oracle."""
+    N, d = 200, 64
+    rng = np.random.default_rng(B)
+    k_len = rng.integers(-3, N + 40, size=B).tolist()
+    k_len[0], k_len[-1] = 0, N
+    q, k, v = rand_inputs(B, 1, N, d, seed=900 + B)
+    check_case(q, k, v, False, 1.0 / math.sqrt(d), k_len=k_len)
+
+
 # ------------------------------------------------------------ grouped key/value heads
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("H_kv", [1, 2, 4])

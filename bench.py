@@ -43,7 +43,7 @@ from exact_io_aware_52_b200 import workloads  # noqa: E402
 DEFAULT_WORKLOAD = 4  # long-context causal B1 H32 N16384 d128: the tensor-bound headline
 METRIC = "attention fwd TFLOP/s (bf16, 1xB200) and % of dense BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["fa_fwd_kernel.cuh", "sm100_ptx.cuh"]  # device code of the d <= 128 kernel (default record)
+KERNEL_SOURCES = ["fa_fwd_kernel.cuh", "fa_softmax_row.cuh", "sm100_ptx.cuh"]  # device code of the d <= 128 kernel
 # Dense bf16 tensor FLOPs per SM per clock of tcgen05 kind::f16 (one 128x128x128
 # product group every 512 cycles); times the SM count and the sampled SM clock it
 # gives the clock-derived dense peak, the second denominator of every fraction.
@@ -624,6 +624,7 @@ def measure_per_config(args, local, peaks, num_sms):
             "tflops": tf, "tflops_p10_time": flops / (st["p10"] * 1e-3) / 1e12,
             "tflops_p90_time": flops / (st["p90"] * 1e-3) / 1e12,
             "frac": tf / peak, "frac_of_burst": tf / burst, "frac_of_sustained": tf / sustained,
+            "algorithmic_bytes": algorithmic_bytes(w, k_len), "traffic": measured_traffic(wid),
             "clocks": clocks,
         }
         if clocks and clocks.get("sm_mhz"):

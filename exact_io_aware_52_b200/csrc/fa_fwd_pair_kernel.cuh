@@ -286,6 +286,9 @@ __device__ __forceinline__ void load_role(const FwdParams &p, const CUtensorMap 
     const uint64_t to = p.timeout_ns;
     const uint32_t q_full0 = cluster_addr(&bars[C::kBarQFull], 0);
     uint32_t tq = 0, gk = 0, gv = 0;
+    // test only: the K load (ring position) the first pair never issues, in
+    // both CTAs, so that no copy is ever in flight toward it
+    const uint32_t drop = ((blockIdx.x >> 1) == 0 && p.drop_load > 0) ? (uint32_t)(p.drop_load - 1) : 0xFFFFFFFFu;
     bool ok = true;
     for (int k = 0; ok; ++k) {
         const int t = pair_unit(p, k);
@@ -307,12 +310,14 @@ __device__ __forceinline__ void load_role(const FwdParams &p, const CUtensorMap 
                     ok = false;
                     break;
                 }
-                if (rank == 0) mbar_arrive_expect_tx(&bars[C::kBarKFull + st], 2 * C::kKBytes);
-                const uint32_t full0 = cluster_addr(&bars[C::kBarKFull + st], 0);
+                if (gk != drop) {
+                    if (rank == 0) mbar_arrive_expect_tx(&bars[C::kBarKFull + st], 2 * C::kKBytes);
+                    const uint32_t full0 = cluster_addr(&bars[C::kBarKFull + st], 0);
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    tma_load_3d_pair(sK + st * C::kKBytes + c * (64 * 128), tm_k64, full0, c * 64,
-                                     kt * BN + 64 * (int)rank, u.bh_kv);
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_3d_pair(sK + st * C::kKBytes + c * (64 * 128), tm_k64, full0, c * 64,
+                                         kt * BN + 64 * (int)rank, u.bh_kv);
+                }
                 ++gk;
             }
             {
@@ -334,7 +339,7 @@ __device__ __forceinline__ void load_role(const FwdParams &p, const CUtensorMap 
     const uint32_t nk = gk < (uint32_t)C::kKStages ? gk : (uint32_t)C::kKStages;
     for (uint32_t i = 0; i < nk; ++i) {
         const uint32_t g = gk - 1 - i;
-        mbar_wait_drain(&bars[C::kBarKFull + g % C::kKStages], (g / C::kKStages) & 1);
+        if (g != drop) mbar_wait_drain(&bars[C::kBarKFull + g % C::kKStages], (g / C::kKStages) & 1);
     }
     const uint32_t nv = gv < (uint32_t)C::kVStages ? gv : (uint32_t)C::kVStages;
     for (uint32_t i = 0; i < nv; ++i) {

@@ -14,11 +14,13 @@
 //     reads half of every K and V tile (the tensor cores exchange the halves);
 //   * per CTA, TMEM holds two score buffers S_0, S_1 (consecutive key tiles),
 //     the output accumulator O and the probabilities P in columns of their
-//     own: S_X K_{j+2}^T may be issued as soon as the softmax has read S(j),
+//     own: Q K_{j+2}^T may be issued as soon as the softmax has read S(j),
 //     and the softmax of tile j+1 never waits for the P V of tile j;
 //   * each query row is shared by two softmax warps on one SM sub-partition,
 //     one per 64-key half of the tile, which exchange their row maxima (and,
-//     at the end of a unit, their sums) through shared memory.
+//     at the end of a unit, their sums) through shared memory; each warp
+//     reads key tile j+1 and posts its half maximum before it computes the
+//     exponentials of tile j, so the exchange overlaps them.
 //
 // TMEM (each CTA, 512 columns allocated as a pair): S_0 [0,128), S_1
 // [128,256), O [256,384), P [384,448) (bf16 pairs).  Warps 0-7 softmax (warp
@@ -135,12 +137,13 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         if (p.k_len) lim = min(max(__ldg(p.k_len + u.b), 0), p.Nk);
         if (p.causal) lim = min(lim, row + 1 + (p.Nk - p.N));
         RowState st;
-        for (int j = 0; j < u.nmax; ++j, ++gs) {
-            const uint32_t buf = gs & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[C::kBarSFull + buf], (gs >> 1) & 1, abort_flag, to));
-            if (!ok) break;
+        // S half-row of key tile j (score tile g overall) into s, its S buffer
+        // released, masked, and this half's maximum posted to the partner warp
+        auto read_half = [&](uint32_t g, int j, float (&s)[64]) -> bool {
+            const uint32_t buf = g & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[C::kBarSFull + buf], (g >> 1) & 1, abort_flag, to)))
+                return false;
             tc_fence_after();
-            float s[64];
             const uint32_t t_s = tmem + lane_off + kColS + 128u * buf + 64u * h;
             tmem_ld32f(t_s, s);
             tmem_ld32f(t_s + 32, s + 32);
@@ -149,24 +152,31 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(s_free0[buf]);  // S_buf may take the key tile after next
-            // masking step on this half's 64 keys, then the row maximum of both halves
-            const int kv0 = (u.lo + j) * BN + 64 * h;
+            const int kv0 = (u.lo + j) * BN + 64 * h;  // masking step on this half's 64 keys
             if (kv0 + 64 > lim) mask_scores<0>(s, kv0, lim);
-            const float m_half = max64(s) * p.scale_log2;
-            xmax[(gs & 1) * 2 * BM + h * BM + r] = m_half;
-            if (!(ok = exchange(&bars[C::kBarXMax + wq], gs))) break;
+            xmax[(g & 1) * 2 * BM + h * BM + r] = max64(s) * p.scale_log2;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[C::kBarXMax + wq]);
+            return true;
+        };
+        // key tile j from `cur`: the row maximum of both halves, the reference
+        // update, the next tile read into `nxt` (its maximum travels to the
+        // partner while this tile's exponentials run), then P and the sums
+        auto tile = [&](float (&cur)[64], float (&nxt)[64], int j) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[C::kBarXMax + wq], gs & 1, abort_flag, to))) return false;
             const float m_new = fmaxf(xmax[(gs & 1) * 2 * BM + r], xmax[(gs & 1) * 2 * BM + BM + r]);
             float alpha;
             const bool resc = update_reference(st, j, m_new, p.tau, alpha);
+            if (j + 1 < u.nmax && !read_half(gs + 1, j + 1, nxt)) return false;
             if (__any_sync(0xffffffffu, resc)) {  // O (this half's 64 columns) *= alpha once P V(j-1) is done
-                if (!(ok = ensure_pv(gs))) break;
+                if (!ensure_pv(gs)) return false;
                 tc_fence_after();
                 rescale_o_row<64>(t_o, alpha);
             }
             uint32_t pk[32];
             float2 ls = make_float2(0.f, 0.f);
-            exp_half_p<0>(s, p.scale_log2, -st.m_ref, pk, ls);
-            if (!(ok = ensure_pv(gs))) break;  // P V(j-1) has read P
+            exp_half_p<0>(cur, p.scale_log2, -st.m_ref, pk, ls);
+            if (!ensure_pv(gs)) return false;  // P V(j-1) has read P
             tc_fence_after();
             tmem_st32(t_p, pk);
             tmem_st_wait();
@@ -178,6 +188,14 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
 #pragma unroll
             for (int i = 0; i < 32; ++i) b4[i & 3] = add_bf16x2_to(b4[i & 3], pk[i]);
             st.lr += (b4[0] + b4[1]) + (b4[2] + b4[3]);
+            ++gs;
+            return true;
+        };
+        float sa[64], sb[64];  // two score buffers in registers, alternating by key tile
+        ok = read_half(gs, 0, sa);
+        for (int j = 0; j < u.nmax && ok; j += 2) {
+            ok = tile(sa, sb, j);
+            if (ok && j + 1 < u.nmax) ok = tile(sb, sa, j + 1);
         }
         if (ok) ok = ensure_pv(gs);  // every product of this unit
         if (ok) {  // both halves' sums, added in the same order by both
@@ -253,7 +271,13 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
         if (!ok) break;
         if (n <= 2) tc_commit_pair(&bars[C::kBarQEmpty], 3);
         for (int j = 0; j < n; ++j) {
-            // O (+)= P V for key tile j, then the scores of key tile j + 2
+            // the scores of key tile j + 2 (their S buffer is free once the
+            // softmax has read tile j, which it does while still working on
+            // tile j - 1), then O (+)= P V for key tile j
+            if (j + 2 < n) {
+                if (!(ok = issue_qk())) break;
+                if (j + 2 == n - 1) tc_commit_pair(&bars[C::kBarQEmpty], 3);
+            }
             if (!mbar_wait(&bars[C::kBarPFull], gp & 1, abort_flag, to)) { ok = false; break; }
             if (j == 0 && tl > 0 && !mbar_wait(&bars[C::kBarOFree], (tl - 1) & 1, abort_flag, to)) { ok = false; break; }
             const uint32_t vst = gv % C::kVStages;
@@ -264,10 +288,6 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
             tc_commit_pair(&bars[C::kBarVEmpty + vst], 3);
             ++gv;
             ++gp;
-            if (j + 2 < n) {
-                if (!(ok = issue_qk())) break;
-                if (j + 2 == n - 1) tc_commit_pair(&bars[C::kBarQEmpty], 3);
-            }
         }
         ++tl;
     }
@@ -394,8 +414,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp < pair::kSoftmaxWarps) {
+        setmaxnreg_inc<kSoftmaxRegs>();
         if (!pair::softmax_role<O_BF16>(p, bars, abort_flag, smem, tmem, rank, warp, lane)) record_timeout(p);
-    } else if (warp == pair::kMmaWarp) {
+    } else {
+        setmaxnreg_dec<kControlRegs>();
+    }
+    if (warp == pair::kMmaWarp) {
         if (lane == 0 && rank == 0) {
             if (!pair::mma_role(p, bars, abort_flag, tmem, smem_u32(sQ), smem_u32(sK), smem_u32(sV)))
                 record_timeout(p);

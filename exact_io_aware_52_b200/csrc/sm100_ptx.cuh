@@ -528,9 +528,13 @@ __device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (possibly in the
-// other CTA of the pair), releasing this thread's prior writes cluster-wide.
+// other CTA of the pair), with the default (CTA-scope release) semantics: the
+// ordering the callers need is that of their tcgen05 loads and stores, which
+// tcgen05.fence::before_thread_sync before the arrive and
+// tcgen05.fence::after_thread_sync after the wait provide; a cluster-scope
+// release would add a full memory fence to every arrival.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
 
 // TMA tile load into this CTA's shared memory whose completion (transaction

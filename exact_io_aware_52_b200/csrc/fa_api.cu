@@ -17,7 +17,6 @@
 #include "fa_combine_kernel.cuh"
 #include "fa_fwd_d256_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
-#include "fa_fwd_pair_kernel.cuh"
 
 namespace {
 
@@ -38,17 +37,12 @@ constexpr int kSchedWords = 4;
 static __device__ __align__(16) uint32_t g_sched[kSchedWords * kSchedSlots];
 std::atomic<uint32_t> g_sched_next{0};
 
-// d = 128 with bf16 inputs on CTA pairs (fa_fwd_pair_kernel.cuh) instead of
-// the one-CTA two-tile kernel.
-constexpr bool kUsePairD128 = false;
-
 struct DeviceInfo {
     bool probed = false;
     bool supported = false;
     int num_sms = 0;
     uint32_t *sched = nullptr;  // g_sched on this device
     bool attr_set[4][2] = {};  // [d = 64, 128, 256, 128 with E4M3 inputs][bf16 out]
-    bool pair_attr_set[2] = {};  // pair kernel [bf16 out]
     bool bwd_attr_set[2] = {};  // backward kernel, [d == 128]
 };
 
@@ -225,43 +219,6 @@ fa_status launch(const fa::FwdParams &kp, DeviceInfo &di, int grid, cudaStream_t
         }
     }
     kern<<<grid, threads, smem, stream>>>(kp);
-    return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-// d = 128, bf16 inputs, on CTA pairs: a static snake order of units over
-// min(units, SMs / 2) pairs; K is read through a second map whose boxes are
-// one CTA's 64 keys.
-template <bool BF16>
-fa_status launch_pair(const fa::FwdParams &kp, const void *k, int BH_kv, int n_k, DeviceInfo &di, cudaStream_t stream) {
-    fa::PairParams pp;
-    std::memset(&pp, 0, sizeof pp);
-    pp.p = kp;
-    pp.p.dynamic = 0;
-    pp.p.sort_b = 0;
-    {
-        cuuint64_t dims[3] = {(cuuint64_t)128, (cuuint64_t)n_k, (cuuint64_t)BH_kv};
-        cuuint64_t strides[2] = {(cuuint64_t)128 * 2, (cuuint64_t)n_k * 128 * 2};
-        cuuint32_t box[3] = {64, 64, 1};
-        cuuint32_t estr[3] = {1, 1, 1};
-        if (g_encode(&pp.tm_k64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return FA_ERR_CUDA;
-    }
-    auto kern = fa::fa_fwd_pair_kernel<BF16>;
-    const int smem = fa::pair::PCfg::kSmemBytes;
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        bool &set = di.pair_attr_set[BF16];
-        if (!set) {
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-                return FA_ERR_CUDA;
-            set = true;
-        }
-    }
-    int pairs = di.num_sms / 2;
-    if (pp.p.n_units < pairs) pairs = pp.p.n_units;
-    kern<<<2 * pairs, fa::pair::kThreads, smem, stream>>>(pp);
     return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -501,15 +458,6 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     const int grid = kp.n_units < di->num_sms ? kp.n_units : di->num_sms;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = p->o_dtype == FA_O_BF16;
-    if (kUsePairD128 && p->d == 128 && !e4m3_in(p) && di->num_sms >= 2) {
-        if (sp.splits > 1) {
-            if ((st = launch_pair<false>(kp, p->k, p->B * H_kv, n_k_map, *di, s)) != FA_OK) return st;
-            return bf16 ? launch_combine_d<true>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)
-                        : launch_combine_d<false>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s);
-        }
-        return bf16 ? launch_pair<true>(kp, p->k, p->B * H_kv, n_k_map, *di, s)
-                    : launch_pair<false>(kp, p->k, p->B * H_kv, n_k_map, *di, s);
-    }
     if (sp.splits > 1) {  // the split pass always writes fp32 partials; the merge writes the output type
         if ((st = launch_d<false>(p->d, e4m3_in(p), kp, *di, grid, s)) != FA_OK) return st;
         return bf16 ? launch_combine_d<true>(p->d, o_part, lse_part, p->o, p->lse, sp.splits, rows, di->num_sms, s)

@@ -6,7 +6,6 @@
 //     in shared memory;
 //   * the same two products with E4M3 operands (tcgen05.mma kind::f8f6f4),
 //     P rounded to E4M3 and packed four per TMEM column by the kernel's packer;
-//   * both products as one CTA-pair (cta_group::2) product of 256 rows;
 //   * the bounded mbarrier wait running out on a barrier nobody arrives at.
 // They use exactly the descriptor builders and MMA issue blocks of the kernel.
 #include <cuda.h>
@@ -339,108 +338,6 @@ __global__ void k_mma_e4m3_ts(const __grid_constant__ SelfParams sp) {
 }
 
 // ---------------------------------------------------------------------------
-// CTA pair (a cluster of two CTAs): S[256][128] = A[256][128] B[128][128]^T and
-// O[256][128] = P[256][128] V[128][128], each one tcgen05 cta_group::2 product
-// issued by CTA 0.  CTA r holds rows [128 r, 128 r + 128) of A, P, S and O,
-// keys [64 r, 64 r + 64) of B (K-major) and value columns [64 r, 64 r + 64) of
-// V (MN-major); both CTAs' operand loads complete on CTA 0's barrier.
-struct PairParams {
-    CUtensorMap ta, tb, tv;  // A [256][128] box {64, 128}; B [128][128] box {64, 64}; V [128][128] box {64, 128}
-    const uint16_t *p;       // P [256][128] bf16
-    float *s, *o;            // [256][128] fp32
-    int32_t *status;
-};
-
-__global__ void __cluster_dims__(2, 1, 1) k_mma_pair(const __grid_constant__ PairParams sp) {
-    extern __shared__ uint8_t raw_smem[];
-    uint8_t *smem = raw_smem + ((1024u - (smem_u32(raw_smem) & 1023u)) & 1023u);
-    uint8_t *sA = smem;          // two 64-column blocks of 128 rows (16 KB each)
-    uint8_t *sB = smem + 32768;  // two 64-column blocks of 64 rows (8 KB each)
-    uint8_t *sV = smem + 49152;  // one 64-column block of 128 key rows (16 KB)
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 65536);  // [0] operands, [1] S done, [2] O done
-    uint32_t *slot = reinterpret_cast<uint32_t *>(smem + 65536 + 64);
-    int *abort_flag = reinterpret_cast<int *>(smem + 65536 + 68);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_rank();
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc_pair(slot, 512);
-        tmem_relinquish_pair();
-    }
-    tc_fence_before();
-    cluster_sync();  // barriers initialised and TMEM allocated in both CTAs
-    tc_fence_after();
-    const uint32_t tmem = *slot;
-    const uint32_t colS = 0, colO = 128, colP = 256;
-    const int row = warp * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    {  // this CTA's P rows into its TMEM, two bf16 per column
-        const uint32_t *prow = reinterpret_cast<const uint32_t *>(sp.p + (size_t)(128 * rank + row) * 128);
-        uint32_t r0[32], r1[32];
-        for (int c = 0; c < 32; ++c) {
-            r0[c] = prow[c];
-            r1[c] = prow[32 + c];
-        }
-        tmem_st32(tmem + lane_off + colP, r0);
-        tmem_st32(tmem + lane_off + colP + 32, r1);
-        tmem_st_wait();
-    }
-    const uint32_t full0 = cluster_addr(&bars[0], 0);
-    if (threadIdx.x == 0 && rank == 0) mbar_arrive_expect_tx(&bars[0], 2 * (32768 + 16384 + 16384));
-    tc_fence_before();
-    cluster_sync();  // P in both TMEMs; CTA 0's operand barrier expects both CTAs' bytes
-    tc_fence_after();
-    if (threadIdx.x == 0) {
-        for (int c = 0; c < 2; ++c) {
-            tma_load_3d_pair(sA + c * 16384, &sp.ta, full0, c * 64, 128 * (int)rank, 0);
-            tma_load_3d_pair(sB + c * 8192, &sp.tb, full0, c * 64, 64 * (int)rank, 0);
-        }
-        tma_load_3d_pair(sV, &sp.tv, full0, 64 * (int)rank, 0, 0);
-    }
-    if (rank == 0 && threadIdx.x == 0) {
-        if (mbar_wait(&bars[0], 0, abort_flag, kTimeoutNs)) {
-            tc_fence_after();
-            mma2_ss_k128_b8k(tmem + colS, sw128_desc(smem_u32(sA), 16, 1024), sw128_desc(smem_u32(sB), 16, 1024),
-                             idesc_bf16_f32(256, 128, false), 0u);
-            tc_commit_pair(&bars[1], 3);
-            mma2_ts_k128(tmem + colO, tmem + colP, sw128_desc(smem_u32(sV), 16384, 1024),
-                         idesc_bf16_f32(256, 128, true), 0u);
-            tc_commit_pair(&bars[2], 3);
-        }
-    }
-    __syncwarp();
-    bool ok = mbar_wait(&bars[1], 0, abort_flag, kTimeoutNs) && mbar_wait(&bars[2], 0, abort_flag, kTimeoutNs);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-        tc_fence_after();
-        const size_t out_row = (size_t)(128 * rank + row) * 128;
-        for (int ch = 0; ch < 4; ++ch) {
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_off + colS + ch * 32, r);
-            tmem_ld_wait();
-            tmem_reg_fence(r);
-            for (int c = 0; c < 32; ++c) sp.s[out_row + ch * 32 + c] = __uint_as_float(r[c]);
-            tmem_ld32(tmem + lane_off + colO + ch * 32, r);
-            tmem_ld_wait();
-            tmem_reg_fence(r);
-            for (int c = 0; c < 32; ++c) sp.o[out_row + ch * 32 + c] = __uint_as_float(r[c]);
-        }
-    } else {
-        set_status(sp.status, 5);
-    }
-    tc_fence_before();
-    cluster_sync();  // both CTAs are done with the pair's TMEM and barriers
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc_pair(tmem, 512);
-    }
-}
-
-// ---------------------------------------------------------------------------
 // A wait on a barrier that nothing ever arrives at must give up after the
 // limit and report it, leaving the context usable.
 __global__ void k_wait_timeout(int32_t *status, uint64_t timeout_ns) {
@@ -477,12 +374,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
     return fn;
 }
 
-int make_map(CUtensorMap *m, const void *base, int rows, int cols, int box_rows = 128) {
+int make_map(CUtensorMap *m, const void *base, int rows, int cols) {
     auto enc = encoder();
     if (!enc) return 4;
     cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, 1};
     cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)rows * cols * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t box[3] = {64, 128, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -585,23 +482,6 @@ int fa_selftest_exp2_poly(const float *x, float *y, int n, void *stream) {
     if (n < 0 || (n & 1)) return 1;
     if (n == 0) return 0;
     k_exp2_poly<<<64, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
-    return finish(stream);
-}
-
-int fa_selftest_mma_pair(const void *a, const void *b, const void *p, const void *v, float *s, float *o,
-                         int32_t *status, void *stream) {
-    if (!a || !b || !p || !v || !s || !o || !status) return 1;
-    PairParams sp;
-    std::memset(&sp, 0, sizeof sp);
-    if (make_map(&sp.ta, a, 256, 128) || make_map(&sp.tb, b, 128, 128, 64) || make_map(&sp.tv, v, 128, 128))
-        return 4;
-    sp.p = static_cast<const uint16_t *>(p);
-    sp.s = s;
-    sp.o = o;
-    sp.status = status;
-    const int smem = 65536 + 128 + 1024;
-    if (cudaFuncSetAttribute(k_mma_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 4;
-    k_mma_pair<<<2, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(sp);
     return finish(stream);
 }
 

@@ -501,120 +501,4 @@ __device__ __forceinline__ float add_bf16x2_to(float acc, uint32_t u) {
 __device__ __forceinline__ float bf16x2_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16x2_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
-// ---------------------------------------------------------------- CTA pairs
-// A cluster of two CTAs on two SMs whose tensor cores run one product of
-// M = 256 rows together (tcgen05 cta_group::2): each CTA holds half of A
-// (its 128 rows) and half of B (N / 2 columns) in its own shared memory, and
-// its 128 rows of D in its own TMEM.  One thread of the pair's first CTA
-// issues the products.
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Every thread of both CTAs: release this CTA's prior writes to the cluster
-// and wait until every thread of the cluster has arrived.
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// The shared::cluster address of the same shared-memory location in CTA `rank`.
-__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-
-// Arrive on an mbarrier given by its shared::cluster address (possibly in the
-// other CTA of the pair), with the default (CTA-scope release) semantics: the
-// ordering the callers need is that of their tcgen05 loads and stores, which
-// tcgen05.fence::before_thread_sync before the arrive and
-// tcgen05.fence::after_thread_sync after the wait provide; a cluster-scope
-// release would add a full memory fence to every arrival.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
-    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
-}
-
-// TMA tile load into this CTA's shared memory whose completion (transaction
-// bytes) is signalled on an mbarrier of the pair's first CTA.
-__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster_addr, int c0,
-                                                 int c1, int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
-// Paired TMEM allocation: one warp of each CTA of the pair (the same warp
-// index in both) allocates the same columns in both SMs.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// Arrive once on the mbarrier at the same shared-memory offset in each CTA of
-// `cta_mask` (bit r: cluster rank r) when every pair product this thread has
-// issued is complete.
-__device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t cta_mask) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_u32(bar)),
-        "h"(cta_mask)
-        : "memory");
-}
-
-// Pair product S (+)= A B^T over K = 128: A (each CTA's 128 rows) and B (each
-// CTA's N / 2 rows) K-major, 128-byte swizzled, two 64-element column blocks
-// each; A's blocks `a_block` bytes apart, B's `b_block` bytes apart (in
-// 16-byte units in the macro below: 1024 = 16 KB, 512 = 8 KB).
-#define FA_SS2_STEP(OA, OB)                                  \
-    "add.s64 da, %1, " #OA ";\n\t"                           \
-    "add.s64 db, %2, " #OB ";\n\t"                           \
-    "tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %3, pt;\n\t"
-__device__ __forceinline__ void mma2_ss_k128_b8k(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-    // A blocks 16 KB apart (128 rows), B blocks 8 KB apart (64 rows)
-    asm volatile(
-        "{\n\t.reg .b64 da, db;\n\t.reg .pred p, pt;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "setp.eq.u32 pt, 1, 1;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t"
-        FA_SS2_STEP(2, 2) FA_SS2_STEP(4, 4) FA_SS2_STEP(6, 6)
-        FA_SS2_STEP(1024, 512) FA_SS2_STEP(1026, 514) FA_SS2_STEP(1028, 516) FA_SS2_STEP(1030, 518)
-        "}" ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-#undef FA_SS2_STEP
-
-// Pair product O (+)= P V over 128 keys: P in each CTA's TMEM (its 128 rows,
-// two bf16 per column), V (each CTA's N / 2 columns) MN-major in shared
-// memory, 16 key rows of 128 bytes per step.
-#define FA_TS2_STEP(TA, DB)                                  \
-    "add.u32 ta, %1, " #TA ";\n\t"                           \
-    "add.s64 db, %2, " #DB ";\n\t"                           \
-    "tcgen05.mma.cta_group::2.kind::f16 [%0], [ta], db, %3, pt;\n\t"
-__device__ __forceinline__ void mma2_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t.reg .pred p, pt;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "setp.eq.u32 pt, 1, 1;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t"
-        FA_TS2_STEP(8, 128) FA_TS2_STEP(16, 256) FA_TS2_STEP(24, 384) FA_TS2_STEP(32, 512)
-        FA_TS2_STEP(40, 640) FA_TS2_STEP(48, 768) FA_TS2_STEP(56, 896)
-        "}" ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-#undef FA_TS2_STEP
-
 }  // namespace fa

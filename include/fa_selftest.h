@@ -56,15 +56,6 @@ FA_SELFTEST_EXPORT int fa_selftest_mma_e4m3_ts(const float *p, const void *v, fl
  * "Calculo de Softmax en linea"); inputs below -127 give +0. */
 FA_SELFTEST_EXPORT int fa_selftest_exp2_poly(const float *x, float *y, int n, void *stream);
 
-/* The CTA-pair form of both products (a cluster of two CTAs on two SMs, one
- * tcgen05 cta_group::2 product of 256 rows each): s[256][128] (fp32) =
- * a[256][128] * b[128][128]^T and o[256][128] (fp32) = p[256][128] *
- * v[128][128], all inputs bf16 row-major; CTA r holds rows [128 r, 128 r +
- * 128) of a and p, keys [64 r, 64 r + 64) of b and value columns
- * [64 r, 64 r + 64) of v. */
-FA_SELFTEST_EXPORT int fa_selftest_mma_pair(const void *a, const void *b, const void *p, const void *v, float *s,
-                                            float *o, int32_t *status, void *stream);
-
 /* Wait on a barrier nothing arrives at, with a limit of timeout_ms; the wait
  * must give up and store 5 in *status. */
 FA_SELFTEST_EXPORT int fa_selftest_wait_timeout(int32_t *status, uint32_t timeout_ms, void *stream);

@@ -142,22 +142,3 @@ def test_polynomial_exp2_error_bound():
     assert torch.equal(yy[ints], ref[ints])
     assert (yy[~live].abs() <= 1e-43).all()
 
-
-def test_cta_pair_products_match_matmul():
-    """The CTA-pair (cta_group::2) form of both products: one 256-row Q K^T
-    and one 256-row P V, each CTA holding its 128 rows of A and P, its 64 keys
-    of B and its 64 value columns of V, equal the float64 products."""
-    lib = fb.load_selftest()
-    g = torch.Generator().manual_seed(321)
-    a = torch.randn(256, 128, generator=g).to(torch.bfloat16)
-    b = torch.randn(128, 128, generator=g).to(torch.bfloat16)
-    p = torch.rand(256, 128, generator=g).to(torch.bfloat16)
-    v = torch.randn(128, 128, generator=g).to(torch.bfloat16)
-    s = torch.full((256, 128), float("nan"), device=_dev())
-    o = torch.full((256, 128), float("nan"), device=_dev())
-    st = _status()
-    ad, bd, pd, vd = (t.to(_dev()) for t in (a, b, p, v))
-    assert lib.fa_selftest_mma_pair(_p(ad), _p(bd), _p(pd), _p(vd), _p(s), _p(o), _p(st), None) == 0
-    assert st.item() == 0
-    np.testing.assert_allclose(s.cpu().double().numpy(), (a.double() @ b.double().T).numpy(), rtol=0, atol=2e-4)
-    np.testing.assert_allclose(o.cpu().double().numpy(), (p.double() @ v.double()).numpy(), rtol=0, atol=2e-4)

@@ -360,8 +360,8 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) 
 // ------------------------------------------------------------------ softmax
 // One warpgroup, query tile x; thread owns row (warp % 4) * 32 + lane.
 // E4M3 probabilities are taken relative to m_ref - kF8Shift (so that they lie
-// in (0, 2^8] with eager rescaling, inside E4M3's normal range down to 2^-14
-// of the row maximum).
+// in (0, 2^(8 + tau)], tau <= 0.75: below E4M3's largest value 448, and
+// normal in E4M3 down to 2^-14 of the reference).
 constexpr float kF8Shift = 8.f;
 
 template <int D, bool O_BF16, bool F8>
@@ -484,9 +484,9 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         tc_fence_after();
         // a row whose allowed keys all lie outside this unit's key range (key
         // splits) has nothing summed: O = 0, lse = -inf for it.  E4M3: O over
-        // the unrounded sum (with eager rescaling the row maximum's weight 2^8
-        // is exact in E4M3, so the rounded and unrounded sums differ only by
-        // the unbiased rounding of the smaller weights)
+        // the unrounded sum (the rounded and unrounded sums differ only by the
+        // unbiased roundings of the weights, each at most 2^-4 relative for
+        // the large ones)
         if constexpr (C::kStageO && !O_BF16) {
             // the warp's 32 rows are consecutive output rows starting at lane 0's
             const size_t first_row_id = row_id - lane;

@@ -3,14 +3,17 @@
 With E4M3 inputs the kernel computes Q K^T exactly up to fp32 accumulation
 (a product of two E4M3 values has at most 8 significant bits), but rounds the
 probabilities to E4M3 before the product with V.  It takes them relative to
-the running row maximum m minus 8 (log2 units) with eager rescaling, so the
-row maximum's weight is 2^8, exact in E4M3, and each weight p'_j = 2^(8 + x_j
-- m) <= 2^8 is rounded either relatively (|dp| <= u p', u = 2^-4, three
-mantissa bits, for p' >= 2^-6, E4M3's smallest normal) or absolutely
+a reference r minus 8 (log2 units) that trails the running row maximum by at
+most tau (0.75, or 0 with eager rescaling): each weight 2^(8 + x_j - r) <=
+2^8.75 < 448 is rounded either relatively (|dp| <= u p, u = 2^-4, three
+mantissa bits, for weights >= 2^-6, E4M3's smallest normal) or absolutely
 (|dp| <= 2^-10, half the subnormal spacing 2^-9, below it).  A weight taken
-while the running maximum was smaller is only larger at rounding time and is
-then scaled down exactly, so the same two cases hold in final units.  O is
-divided by the unrounded sum L' = sum_j p'_j, hence
+while the reference was smaller is only larger at rounding time and is then
+scaled down exactly.  In units of the true row maximum m (p'_j = 2^(8 + x_j -
+m)) the final reference lies delta, 0 <= delta <= tau, below m: the
+absolutely rounded weights are a subset of those with p'_j < 2^-6, and their
+error over the sum is at most 2^-10 / (2^delta L') <= 2^-10 / L'.  O is
+divided by the unrounded sum, which is L' = sum_j p'_j in units of m, hence
 
     |O_kernel - O| = |sum_j dp_j v_j| / L'
                   <= u sum_j w_j |v_j| + 2^-10 / L' * sum_{j: p'_j < 2^-6} |v_j|

@@ -14,6 +14,7 @@ import pytest
 import torch
 
 import oracle
+from exact_io_aware_52_b200 import _binding as fb
 from exact_io_aware_52_b200 import workloads
 from tests import fp8_bound
 from tests.gpu_util import TOL_LSE, run_gpu
@@ -34,10 +35,10 @@ def e4m3_inputs(B, H, N, seed, std=1.0, H_kv=None, Nk=None, vstd=1.0):
 
 
 def check_e4m3(q, k, v, causal, scale, descale=(0.0, 0.0, 0.0), k_len=None, rows=None, out_dtype=torch.float32,
-               num_splits=0):
+               num_splits=0, flags=0):
     dq, dk, dv = (x if x > 0 else 1.0 for x in descale)
     o, lse = run_gpu(q, k, v, causal, scale, k_len=k_len, out_dtype=out_dtype, num_splits=num_splits,
-                     descale=descale)
+                     descale=descale, flags=flags)
     sig = float(np.float32(scale * dq * dk))
     kl = None if k_len is None else list(k_len)
     o_ref, lse_ref = oracle.attention_f64(q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16), causal,
@@ -95,11 +96,33 @@ def test_descale_factors():
         check_e4m3(q, k, v, causal, SCALE, descale=(0.5, 2.0, 0.25))
 
 
+@pytest.mark.parametrize("flags", [0, fb.FA_FLAG_EAGER_RESCALE])
 @pytest.mark.parametrize("std", [2.0, 4.0])
-def test_large_logits(std):
+def test_large_logits(std, flags):
     """Peaked rows: a few keys carry the weight, the bound's worst case."""
     q, k, v = e4m3_inputs(1, 4, 2048, seed=3004 + int(std), std=std)
-    print(check_e4m3(q, k, v, True, SCALE))
+    print(check_e4m3(q, k, v, True, SCALE, flags=flags))
+
+
+@pytest.mark.parametrize("flags", [0, fb.FA_FLAG_EAGER_RESCALE])
+def test_slowly_growing_maximum(flags):
+    """Scores that grow along the keys by about 0.4 (head 0) and 1.0 (head 1)
+    natural units per key tile: the row maximum moves on most tiles, often by
+    less than the rescale threshold (weights then reach up to 2^8.75 before
+    rounding) and often by more."""
+    B, H, N = 1, 2, 1024
+    g = torch.Generator().manual_seed(3010 + flags)
+    q = torch.zeros(B, H, N, D)
+    k = torch.zeros(B, H, N, D)
+    q[..., 0] = 1.0
+    q[..., 1] = 0.5
+    k[0, 0, :, 0] = torch.linspace(0.0, 0.4 * N / 128, N)
+    k[0, 1, :, 0] = torch.linspace(0.0, 1.0 * N / 128, N)
+    k[..., 1] = torch.randn(B, H, N, generator=g)
+    v = torch.randn(B, H, N, D, generator=g)
+    q, k, v = (t.to(torch.float8_e4m3fn) for t in (q, k, v))
+    for causal in (False, True):
+        print(check_e4m3(q, k, v, causal, 1.0, flags=flags))
 
 
 @pytest.mark.parametrize("splits", [3, 8])

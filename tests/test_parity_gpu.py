@@ -137,14 +137,38 @@ def test_dominant_key_selects_its_value():
 
 
 # ------------------------------------------------------------ adversarial inputs
-def test_monotone_logits_force_rescale_every_tile():
+@pytest.mark.parametrize("d", [64, 128])
+def test_monotone_logits_force_rescale_every_tile(d):
     """Scores that grow along the keys move the row maximum on every tile."""
-    B, H, N, d = 1, 2, 1024, 64
+    B, H, N = 1, 2, 1024
     q = torch.zeros(B, H, N, d)
     k = torch.zeros(B, H, N, d)
     q[..., 0] = 1.0
     k[..., 0] = torch.linspace(-20, 60, N)
     g = torch.Generator().manual_seed(8)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    for flags in (0, fb.FA_FLAG_EAGER_RESCALE):
+        for causal in (False, True):
+            check_case(q.to(torch.bfloat16), k.to(torch.bfloat16), v, causal, 1.0, flags=flags)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_row_maximum_jumps(d):
+    """Single keys 10, 70 and 130 above the rest (about 14, 101 and 188 in
+    log2 units) in the second, third and fourth key tiles: the row maximum
+    jumps by less than and by more than 64 binary orders on a later tile, so
+    that tile's weights, taken first against the old maximum, are either scaled
+    down or taken again from the scores."""
+    B, H, N = 1, 2, 640
+    g = torch.Generator().manual_seed(17)
+    q = torch.zeros(B, H, N, d)
+    k = torch.zeros(B, H, N, d)
+    q[..., 0] = 1.0
+    q[..., 1] = 0.5
+    k[..., 1] = torch.randn(B, H, N, generator=g)
+    k[:, :, 200, 0] = 10.0
+    k[:, :, 330, 0] = 70.0
+    k[:, :, 500, 0] = 130.0
     v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
     for flags in (0, fb.FA_FLAG_EAGER_RESCALE):
         for causal in (False, True):

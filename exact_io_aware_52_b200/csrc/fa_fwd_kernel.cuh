@@ -448,11 +448,11 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
                 tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
             } else if constexpr (kSep) {
                 exp_half_p<0>(s, p.scale_log2, -st.m_ref, pk0, ls);
-                exp_half_p<1>(s, p.scale_log2, -st.m_ref, pk1, ls);
                 // P_X(j - 1) must have been read by its product before it is replaced
                 if (!(ok = ensure_pv(gs))) break;
                 tc_fence_after();
                 tmem_st32(t_p + 0, pk0);
+                exp_half_p<1>(s, p.scale_log2, -st.m_ref, pk1, ls);
                 tmem_st32(t_p + 32, pk1);
             } else {
                 exp_half_p<0>(s, p.scale_log2, -st.m_ref, pk0, ls);

@@ -139,6 +139,8 @@ def load_selftest():
             lib.fa_selftest_mma_e4m3_ts.argtypes = [vp, vp, vp, vp, vp]
             lib.fa_selftest_exp2_poly.restype = i
             lib.fa_selftest_exp2_poly.argtypes = [vp, vp, i, vp]
+            lib.fa_selftest_mufu_rate.restype = i
+            lib.fa_selftest_mufu_rate.argtypes = [i, i, i, ctypes.POINTER(ctypes.c_double), vp]
             lib.fa_selftest_wait_timeout.restype = i
             lib.fa_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
             _selftest = lib

@@ -362,6 +362,44 @@ __global__ void k_exp2_poly(const float *x, float *y, int n) {
     }
 }
 
+// Exponential-unit rate: every thread runs `iters` passes of 128 exponentials
+// of its own values (MIX = 0: independent ex2 only, summed into 8 chains;
+// MIX = 1: the softmax's mix per pair of keys, one FFMA2, two ex2, one FADD2
+// into 4 chains and one bf16 pack); lane 0 of each warp records the cycles.
+template <int MIX>
+__global__ void k_mufu_rate(float *sink, long long *cycles, int iters) {
+    float s[128];
+#pragma unroll
+    for (int i = 0; i < 128; ++i) s[i] = (threadIdx.x * 0.001f + i) * 0.01f;
+    float m = 0.5f, acc = 0.f;
+    const long long t0 = clock64();
+    for (int it = 0; it < iters; ++it) {
+        if (MIX == 0) {
+            float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < 128; ++c) b[c & 7] += ex2_approx(s[c] - m);
+            acc += ((b[0] + b[1]) + (b[2] + b[3])) + ((b[4] + b[5]) + (b[6] + b[7]));
+        } else {
+            const float2 sl2 = make_float2(1.4426950f, 1.4426950f), nm = make_float2(-m, -m);
+            float2 a[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            uint32_t h = 0;
+#pragma unroll
+            for (int c = 0; c < 128; c += 2) {
+                const float2 xx = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2, nm);
+                const float2 pp = make_float2(ex2_approx(xx.x), ex2_approx(xx.y));
+                a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], pp);
+                h ^= pack_bf16x2(pp.x, pp.y);
+            }
+            acc += (a[0].x + a[1].x) + (a[2].x + a[3].x) + (a[0].y + a[1].y) + (a[2].y + a[3].y) +
+                   __uint_as_float(h & 0x3fffffffu);
+        }
+        m += 1e-7f;
+    }
+    const long long t1 = clock64();
+    sink[blockIdx.x * blockDim.x + threadIdx.x] = acc;
+    if ((threadIdx.x & 31) == 0) cycles[blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)] = t1 - t0;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -483,6 +521,41 @@ int fa_selftest_exp2_poly(const float *x, float *y, int n, void *stream) {
     if (n == 0) return 0;
     k_exp2_poly<<<64, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
     return finish(stream);
+}
+
+int fa_selftest_mufu_rate(int warps_per_subpartition, int mix, int iters, double *cycles_per_pass, void *stream) {
+    if (warps_per_subpartition < 1 || warps_per_subpartition > 8 || (mix != 0 && mix != 1) || iters < 1 ||
+        iters > 100000 || !cycles_per_pass)
+        return 1;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return 4;
+    const int threads = 128 * warps_per_subpartition, warps = sms * (threads / 32);
+    float *sink = nullptr;
+    long long *cyc = nullptr;
+    if (cudaMalloc(&sink, (size_t)sms * threads * sizeof(float)) != cudaSuccess) return 4;
+    if (cudaMalloc(&cyc, (size_t)warps * sizeof(long long)) != cudaSuccess) {
+        cudaFree(sink);
+        return 4;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    for (int rep = 0; rep < 2; ++rep) {  // the first launch warms up
+        if (mix) k_mufu_rate<1><<<sms, threads, 0, st>>>(sink, cyc, iters);
+        else k_mufu_rate<0><<<sms, threads, 0, st>>>(sink, cyc, iters);
+    }
+    int rc = finish(stream);
+    if (rc == 0) {
+        long long *h = new long long[warps];
+        if (cudaMemcpy(h, cyc, (size_t)warps * sizeof(long long), cudaMemcpyDeviceToHost) != cudaSuccess) rc = 4;
+        double sum = 0.0;
+        for (int i = 0; i < warps; ++i) sum += (double)h[i];
+        *cycles_per_pass = sum / warps / iters;
+        delete[] h;
+    }
+    cudaFree(sink);
+    cudaFree(cyc);
+    return rc;
 }
 
 int fa_selftest_wait_timeout(int32_t *status, uint32_t timeout_ms, void *stream) {

@@ -56,6 +56,19 @@ FA_SELFTEST_EXPORT int fa_selftest_mma_e4m3_ts(const float *p, const void *v, fl
  * "Calculo de Softmax en linea"); inputs below -127 give +0. */
 FA_SELFTEST_EXPORT int fa_selftest_exp2_poly(const float *x, float *y, int n, void *stream);
 
+/* Measurement, not a check: the exponential unit's rate as the softmax sees
+ * it.  One CTA per SM, 4 * warps_per_subpartition warps (1..8 per SM
+ * sub-partition); every thread runs `iters` (1..100000) passes of 128
+ * exponentials (mix = 0: independent ex2 only; mix = 1: the softmax's mix of
+ * one FFMA2, two ex2, one FADD2 and one bf16 pack per pair of keys).
+ * *cycles_per_pass (host) receives the mean clock cycles of one warp's pass;
+ * 128 * 32 * warps_per_subpartition / *cycles_per_pass is then the ex2 lanes
+ * per clock one sub-partition delivered.  Allocates and frees two small
+ * device buffers; synchronises `stream`.  Returns 0, 1 for a bad argument,
+ * 4 for a CUDA error. */
+FA_SELFTEST_EXPORT int fa_selftest_mufu_rate(int warps_per_subpartition, int mix, int iters,
+                                             double *cycles_per_pass, void *stream);
+
 /* Wait on a barrier nothing arrives at, with a limit of timeout_ms; the wait
  * must give up and store 5 in *status. */
 FA_SELFTEST_EXPORT int fa_selftest_wait_timeout(int32_t *status, uint32_t timeout_ms, void *stream);

@@ -142,3 +142,22 @@ def test_polynomial_exp2_error_bound():
     assert torch.equal(yy[ints], ref[ints])
     assert (yy[~live].abs() <= 1e-43).all()
 
+
+
+def test_exponential_unit_rate():
+    """Measurement behind the softmax design: one SM sub-partition delivers at
+    most 4 exp2 lanes per clock (16 per SM), and one warp alone gets less of
+    that than two side by side, least with the softmax's own mix of work."""
+    import ctypes
+    lib = fb.load_selftest()
+    rate = {}
+    for mix in (0, 1):
+        for w in (1, 2):
+            c = ctypes.c_double(0.0)
+            assert lib.fa_selftest_mufu_rate(w, mix, 200, ctypes.byref(c), None) == 0
+            rate[mix, w] = 128 * 32 * w / c.value
+    print("exp2 lanes per clock per sub-partition (ex2 only, 1 and 2 warps; softmax mix, 1 and 2 warps):",
+          ", ".join(f"{rate[k]:.2f}" for k in sorted(rate)))
+    assert all(0.0 < r <= 4.2 for r in rate.values()), rate
+    assert rate[0, 2] >= rate[0, 1] and rate[1, 2] >= rate[1, 1], rate
+    assert lib.fa_selftest_mufu_rate(0, 0, 10, ctypes.byref(ctypes.c_double()), None) == 1

@@ -135,6 +135,20 @@ fa_status encode_map_f32(CUtensorMap *map, void *base, int BH, int N, int D) {
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// 3-D map over the fp32 output [planes][N][D] (planes = key splits x B x H),
+// box {32, 32, 1}, 128-byte swizzle: the d = 64 epilogue's TMA stores of one
+// warp's 32 rows, 32 columns per box.  Rows past N are not written.
+fa_status encode_map_o32(CUtensorMap *map, void *base, long long planes, int N, int D) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)planes};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)N * D * 4};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 // Validation that needs no device, except the workspace clause.
 fa_status validate_args(const fa_fwd_params *p) {
     if (!p) return FA_ERR_INVALID_ARGUMENT;
@@ -407,6 +421,9 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
         kp.o = p->o;
         kp.lse = p->lse;
     }
+    // d = 64 bf16 inputs with fp32 output (or fp32 partials): O leaves through TMA stores
+    if (p->d == 64 && !e4m3_in(p) && (sp.splits > 1 || p->o_dtype != FA_O_BF16))
+        if ((st = encode_map_o32(&kp.tm_o, kp.o, (long long)sp.splits * BH, p->N, p->d)) != FA_OK) return st;
     kp.k_len = p->k_len;
     kp.status = p->dev_status;
     kp.B = p->B;

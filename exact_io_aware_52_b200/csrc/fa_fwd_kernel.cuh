@@ -94,6 +94,8 @@ __device__ __forceinline__ uint32_t col_p_sep(uint32_t x) { return 384u + x * 64
 struct FwdParams {
     CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps over [B*H][N][D] (Q) and [B*H_kv][Nk][D] (K, V) bf16;
                                    // box {64, 128, 1}; 128-byte swizzle
+    CUtensorMap tm_o;              // d = 64, fp32 O: 3-D map over o as [n_splits*B*H][N][64] fp32,
+                                   // box {32, 32, 1}, 128-byte swizzle (the epilogue's TMA stores)
     void *o;                       // [n_splits][B, H, N, D] fp32 or bf16 (n_splits > 1: fp32 partials)
     float *lse;                    // [n_splits][B, H, N]
     const int32_t *k_len;          // [B] or nullptr
@@ -133,7 +135,7 @@ struct Cfg {
     static constexpr int kChunkBytes = BM * 128;           // one column block of a 128-row tile
     static constexpr int kTileBytes = BM * D * kElemBytes; // one 128 x D tile
     static constexpr int kKStages = F8 ? 4 : (D == 128) ? 3 : 4;
-    static constexpr int kVStages = F8 ? 4 : (D == 128) ? 2 : 4;
+    static constexpr int kVStages = F8 ? 4 : (D == 128) ? 2 : 3;  // d = 64: a stage gives way to the O stages
     static constexpr int kOffQ = 0;                                   // Q_A, Q_B
     static constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;
@@ -160,13 +162,15 @@ struct Cfg {
     static constexpr int kOffClaimed = kOffAbort + 4;                // scheduler slot claimed (int)
     static constexpr int kOffUnitIds = kOffClaimed + 4;              // [kUnitQueue][4] ints
     static constexpr int kOffBOrder = kOffUnitIds + 16 * kUnitQueue;  // [kSortMaxB] ints
-    // d = 64: per softmax warp a [32][36]-float stage for coalesced O stores
+    // d = 64: per softmax warp D / 32 boxes of [32 rows][32 fp32 columns] in the
+    // 128-byte swizzle, the source of the fp32 O epilogue's TMA stores
     static constexpr bool kStageO = kSepP<D> && !F8;
-    static constexpr int kOffStage = (kOffBOrder + 4 * kSortMaxB + 127) & ~127;  // float4 accesses
-    static constexpr int kSmemUsed = kOffStage + (kStageO ? kSoftmaxWarps * 32 * 36 * 4 : 0);
+    static constexpr int kStageBytes = (D / 32) * 4096;
+    static constexpr int kOffStage = (kOffBOrder + 4 * kSortMaxB + 1023) & ~1023;  // swizzled TMA boxes
+    static constexpr int kSmemUsed = kOffStage + (kStageO ? kSoftmaxWarps * kStageBytes : 0);
     static constexpr int kSmemBytes = kSmemUsed + 1024;  // + slack to align the base to 1024 bytes
     static_assert(kChunkBytes % 1024 == 0 && kTileBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
-    static_assert(kOffStage % 16 == 0, "the O stage is accessed as float4");
+    static_assert(kOffStage % 1024 == 0, "the O stage holds 128-byte-swizzled TMA boxes");
     static_assert(kSmemBytes <= 232448, "shared memory budget of one sm_100 CTA");
     static_assert(2 * kSmemBytes > 233472, "one CTA per SM: TMEM is allocated whole");
 };
@@ -367,7 +371,7 @@ constexpr float kF8Shift = 8.f;
 template <int D, bool O_BF16, bool F8>
 __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
                                              const UnitQueue &uq, uint32_t tmem, int x, int warp, int lane,
-                                             float *stage) {
+                                             uint8_t *stage) {
     using C = Cfg<D, F8>;
     const int row_in_tile = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -385,6 +389,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
     uint32_t gs = 0;  // S tiles of this query tile consumed so far (s_full / p_full phase)
     uint32_t tl = 0;  // units in which this query tile had work (o_final / o_free phase)
     uint32_t pv_known = 0;  // separate P: P_X V products known to be complete
+    bool store_pending = false;  // TMA epilogue (lane 0): a store may still be reading the stage
     // separate P: wait until the first n P_X V products are complete (phases
     // complete in order, and product n cannot start before this thread stores
     // P_X(n), so the parity of phase n - 1 is unambiguous)
@@ -491,8 +496,8 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             // the warp's 32 rows are consecutive output rows starting at lane 0's
             const size_t first_row_id = row_id - lane;
             const int n_valid = min(32, p.N - (row - lane));
-            write_rows_coalesced<D>(t_o, stage, lane, static_cast<float *>(p.o), p.lse, first_row_id, n_valid, st.lr,
-                                    st.m_ref + log2f(st.l));
+            write_rows_tma<D>(t_o, stage, lane, &p.tm_o, row - lane, u.split * p.B * p.H + u.bh, p.lse, first_row_id,
+                              n_valid, st.lr, st.m_ref + log2f(st.l), store_pending);
         } else {
             write_row<D, O_BF16>(t_o, p.o, p.lse, row_id, row_valid, F8 ? st.l : st.lr, F8 ? p.out_scale : 1.f,
                                  st.m_ref - (F8 ? kF8Shift : 0.f) + log2f(st.l));
@@ -500,6 +505,9 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
         tc_fence_before();
         mbar_arrive(o_free);
         ++tl;
+    }
+    if constexpr (C::kStageO && !O_BF16) {
+        if (lane == 0 && store_pending) bulk_wait_group0();  // every O store has completed
     }
     return ok;
 }
@@ -799,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
 
     if (warp < kSoftmaxWarps) {
         setmaxnreg_inc<kSoftmaxRegs>();
-        float *stage = reinterpret_cast<float *>(smem + C::kOffStage) + warp * 32 * 36;
+        uint8_t *stage = smem + C::kOffStage + warp * C::kStageBytes;
         if (!softmax_role<D, O_BF16, F8>(p, bars, abort_flag, uq, tmem, warp >> 2, warp, lane, stage))
             record_timeout(p);
     } else {

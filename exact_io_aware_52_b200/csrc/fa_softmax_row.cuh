@@ -223,40 +223,43 @@ __device__ __forceinline__ void write_row(uint32_t t_o, void *o, float *lse, siz
     if (row_valid) lse[row_id] = empty ? __int_as_float(0xff800000) : lse_log2 * LN2;
 }
 
-// Epilogue of the 32 rows of one warp with coalesced stores (fp32 O): each
-// thread scales its row's D columns and stages them, 32 columns at a time, in
-// the warp's `stage` ([32][36] floats of shared memory, a padded stride that
-// keeps both the row-wise writes and the column-wise reads free of bank
-// conflicts); the warp then writes 4 rows of 32 columns per store instruction
-// (4 cache lines instead of 32 for one row per thread).  `first_row_id` is
-// the output row of lane 0 (the warp's rows are consecutive), `n_valid` how
-// many of the 32 rows exist (rows past N are not written).
+// Epilogue of the 32 rows of one warp through a TMA store (fp32 O): each
+// thread scales its row's D columns and writes them into the warp's stage, D / 32
+// boxes of [32 rows][32 columns] in the 128-byte swizzle of the O tensor map
+// (conflict-free: each 16-byte chunk of a row lands in its own bank group);
+// lane 0 then stores the boxes with one TMA store each and returns at once.
+// `stage` is 1024-byte aligned; `pending` (lane 0) records that an earlier
+// store may still be reading it.  Rows past the head's N are clipped by the
+// tensor map; lse goes out per thread.
 template <int D>
-__device__ __forceinline__ void write_rows_coalesced(uint32_t t_o, float *stage, int lane, float *o, float *lse,
-                                                     size_t first_row_id, int n_valid, float norm, float lse_log2) {
+__device__ __forceinline__ void write_rows_tma(uint32_t t_o, uint8_t *stage, int lane, const CUtensorMap *tm_o,
+                                               int row0, int plane, float *lse, size_t first_row_id, int n_valid,
+                                               float norm, float lse_log2, bool &pending) {
     const float LN2 = 0.69314718055994530942f;
     const bool empty = !(norm > 0.f);
     const float inv_l = empty ? 0.f : 1.f / norm;
+    if (lane == 0 && pending) bulk_wait_group_read0();  // the previous unit's boxes have left the stage
+    __syncwarp();
 #pragma unroll
     for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t r[32];
         tmem_ld32(t_o + ch * 32, r);
         tmem_ld_wait();
         tmem_reg_fence(r);
-        float4 *mine = reinterpret_cast<float4 *>(stage + lane * 36);
+        uint8_t *box = stage + ch * 4096 + lane * 128;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            mine[i] = make_float4(__uint_as_float(r[4 * i + 0]) * inv_l, __uint_as_float(r[4 * i + 1]) * inv_l,
-                                  __uint_as_float(r[4 * i + 2]) * inv_l, __uint_as_float(r[4 * i + 3]) * inv_l);
-        __syncwarp();
+        for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4 *>(box + ((u ^ (lane & 7)) << 4)) =
+                make_float4(__uint_as_float(r[4 * u + 0]) * inv_l, __uint_as_float(r[4 * u + 1]) * inv_l,
+                            __uint_as_float(r[4 * u + 2]) * inv_l, __uint_as_float(r[4 * u + 3]) * inv_l);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the TMA engine
+    __syncwarp();
+    if (lane == 0) {
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-            const int rr = 4 * it + (lane >> 3), c4 = (lane & 7) * 4;
-            if (rr < n_valid)
-                *reinterpret_cast<float4 *>(o + (first_row_id + rr) * D + ch * 32 + c4) =
-                    *reinterpret_cast<const float4 *>(stage + rr * 36 + c4);
-        }
-        __syncwarp();
+        for (int ch = 0; ch < D / 32; ++ch) tma_store_3d(tm_o, stage + ch * 4096, ch * 32, row0, plane);
+        bulk_commit_group();
+        pending = true;
     }
     if (lane < n_valid) lse[first_row_id + lane] = empty ? __int_as_float(0xff800000) : lse_log2 * LN2;
 }

@@ -116,6 +116,17 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap *map, const 
         "r"(c2)
         : "memory");
 }
+// Copy of a shared-memory tile to global memory through a tensor map (TMA
+// store), tracked by the issuing thread's bulk async-group.  Elements of the
+// box outside the tensor are not written.  The innermost coordinate c0 must
+// be a multiple of 16 bytes' worth of elements and no coordinate negative.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group"
+        " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1),
+        "r"(c2)
+        : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until every committed bulk group of this thread has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_group_read0() {

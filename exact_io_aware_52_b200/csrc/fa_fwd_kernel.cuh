@@ -29,10 +29,12 @@
 //   warp 9     TMA producer (one thread): Q_A and Q_B once per unit, K_j and
 //              V_j through separate rings (warps 10-11 idle).
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256, 256+D),
-// O_B [256+D, 256+2D); P_X occupies the first 64 columns of S_X (two bf16 per
-// 32-bit column).
+// O_B [256+D, 256+2D); at d = 128 with bf16 inputs P_X occupies the first 64
+// columns of S_X (two bf16 per 32-bit column); at d = 64 it has columns of its
+// own (kSepP) and with E4M3 inputs it sits in shared memory (kSmemP), and
+// the MMA order is that of the separate-P loop in mma_role.
 //
-// MMA issue order inside a unit, for key tiles j = 1, 2, ...:
+// MMA issue order inside a unit (P over S), for key tiles j = 1, 2, ...:
 //     P_A V_{j-1},  Q_A K_j^T,  P_B V_{j-1},  Q_B K_j^T
 // so the tensor core works on one tile while the other tile's softmax runs.
 // tcgen05.mma operations issued by one thread execute in issue order, which
@@ -79,13 +81,16 @@ constexpr int kStatusSchedBusy = 7;  // FA_ERR_SCHED_BUSY
 // (barrier pv_done, one phase per product).
 template <int D>
 constexpr bool kSepP = (D == 64);
-// The V ring slot of key tile j-1 is released right after the last P_X V_{j-1}
-// product is issued (before Q_B K_j^T) instead of at the end of the step.
-// Measured on B200 (300 launches): E4M3 (B1 H32 N16384 causal) 1.852 ->
-// 1.788 ms; bf16 d = 128 unchanged, d = 64 (B8 H12 N1024 causal) 43.0 ->
-// 44.0 us.  On for E4M3 only.
+// E4M3: P (one byte per key, 16 KB per tile) goes to shared memory instead of
+// over S in TMEM, and P_X V reads it from there (both operands in shared
+// memory); as with separate P columns, Q_X K_{j+1}^T may then run as soon as
+// the softmax has read S_X(j), and the store of the next P waits for P_X V_j.
 template <bool F8>
-constexpr bool kEarlyVRelease = F8;
+constexpr bool kSmemP = F8;
+// S released once read (barrier s_free), each P_X V signalled (pv_done):
+// separate P columns (d = 64) or P in shared memory (E4M3).
+template <int D, bool F8>
+constexpr bool kSepChain = (kSepP<D> && !F8) || kSmemP<F8>;
 
 __device__ __forceinline__ uint32_t col_s(uint32_t x) { return x * 128u; }                  // S_X, P_X
 __device__ __forceinline__ uint32_t col_o(uint32_t x, uint32_t d) { return 256u + x * d; }  // O_X
@@ -139,7 +144,8 @@ struct Cfg {
     static constexpr int kOffQ = 0;                                   // Q_A, Q_B
     static constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-    static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+    static constexpr int kOffP = kOffV + kVStages * kTileBytes;  // P_A, P_B (kSmemP)
+    static constexpr int kOffBar = kOffP + (kSmemP<F8> ? kQTiles * kTileBytes : 0);
     // barrier slots
     static constexpr int kBarQFull = 0;
     static constexpr int kBarQEmpty = 1;
@@ -371,7 +377,7 @@ constexpr float kF8Shift = 8.f;
 template <int D, bool O_BF16, bool F8>
 __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
                                              const UnitQueue &uq, uint32_t tmem, int x, int warp, int lane,
-                                             uint8_t *stage) {
+                                             uint8_t *stage, uint8_t *sP) {
     using C = Cfg<D, F8>;
     const int row_in_tile = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -382,10 +388,10 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
     uint64_t *o_free = &bars[C::kBarOFree + x];
     uint64_t *s_free = &bars[C::kBarSFree + x];
     uint64_t *pv_done = &bars[C::kBarPvDone + x];
-    constexpr bool kSep = kSepP<D> && !F8;
+    constexpr bool kSep = kSepChain<D, F8>;
     const uint32_t t_s = tmem + lane_off + col_s(x);
     const uint32_t t_o = tmem + lane_off + col_o(x, D);
-    const uint32_t t_p = tmem + lane_off + (kSep ? col_p_sep(x) : col_s(x));
+    const uint32_t t_p = tmem + lane_off + ((kSepP<D> && !F8) ? col_p_sep(x) : col_s(x));
     uint32_t gs = 0;  // S tiles of this query tile consumed so far (s_full / p_full phase)
     uint32_t tl = 0;  // units in which this query tile had work (o_final / o_free phase)
     uint32_t pv_known = 0;  // separate P: P_X V products known to be complete
@@ -450,7 +456,15 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
             }
             if constexpr (F8) {
                 exp_e4m3(s, p.scale_log2, kF8Shift - st.m_ref, pk0, ls);
-                tmem_st32(t_s + 0, pk0);  // P overwrites scores already in registers
+                // P_X(j - 1) must have been read by its product before it is replaced
+                if (!(ok = ensure_pv(gs))) break;
+                // this row of P_X: 128 bytes of the K-major tile in the 128-byte swizzle
+                uint8_t *prow = sP + x * C::kTileBytes + row_in_tile * 128;
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<uint4 *>(prow + ((u ^ (row_in_tile & 7)) << 4)) =
+                        make_uint4(pk0[4 * u], pk0[4 * u + 1], pk0[4 * u + 2], pk0[4 * u + 3]);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
             } else if constexpr (kSep) {
                 exp_half_p<0>(s, p.scale_log2, -st.m_ref, pk0, ls);
                 // P_X(j - 1) must have been read by its product before it is replaced
@@ -516,7 +530,7 @@ __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars,
 template <int D, bool F8>
 __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,
                                          const UnitQueue &uq, uint32_t tmem, uint32_t q_addr, uint32_t k_addr,
-                                         uint32_t v_addr) {
+                                         uint32_t v_addr, uint32_t p_addr) {
     using C = Cfg<D, F8>;
     const uint32_t idesc_qk = F8 ? idesc_e4m3_f32(BM, BN, false) : idesc_bf16_f32(BM, BN, false);
     const uint32_t idesc_pv = F8 ? idesc_e4m3_f32(BM, D, true) : idesc_bf16_f32(BM, D, true);
@@ -525,6 +539,7 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
     const uint64_t q_desc = sw128_desc(q_addr, 16, 1024);
     const uint64_t k_desc = sw128_desc(k_addr, 16, 1024);
     const uint64_t v_desc = sw128_desc(v_addr, C::kChunkBytes, 1024);
+    const uint64_t p_desc = sw128_desc(p_addr, 16, 1024);  // P_A, P_B in shared memory (kSmemP), K-major
     uint32_t tq = 0;              // non-empty units (q_full phase)
     uint32_t gk = 0, gv = 0;      // K and V ring positions
     uint32_t gp0 = 0, gp1 = 0;    // P_X V products issued (p_full phase)
@@ -544,19 +559,11 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
     // fresh accumulator, `last` ends the unit for tile X
     auto pv = [&](int x, uint32_t &gpx, uint32_t tlx, uint32_t vslot, bool first, bool last) -> bool {
         const uint64_t vd = v_desc + ((vslot * C::kTileBytes) >> 4);
-        if constexpr (F8) {
-            if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
-            ++gpx;
-            if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
-            tc_fence_after();
-            mma_e4m3_ts_k128(tmem + col_o(x, D), tmem + col_s(x), vd, idesc_pv, first ? 0u : 1u);
-        } else {
-            if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
-            ++gpx;
-            if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
-            tc_fence_after();
-            mma_ts_k128(tmem + col_o(x, D), tmem + col_s(x), vd, idesc_pv, first ? 0u : 1u);
-        }
+        if (!mbar_wait(&bars[C::kBarPFull + x], gpx & 1, abort_flag, to)) return false;
+        ++gpx;
+        if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
+        tc_fence_after();
+        mma_ts_k128(tmem + col_o(x, D), tmem + col_s(x), vd, idesc_pv, first ? 0u : 1u);
         if (last) tc_commit(&bars[C::kBarOFinal + x]);
         return true;
     };
@@ -576,8 +583,12 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
         ++gpx;
         if (first && tlx > 0 && !mbar_wait(&bars[C::kBarOFree + x], (tlx - 1) & 1, abort_flag, to)) return false;
         tc_fence_after();
-        mma_ts_k128(tmem + col_o(x, D), tmem + col_p_sep(x), v_desc + ((vslot * C::kTileBytes) >> 4), idesc_pv,
-                    first ? 0u : 1u);
+        if constexpr (F8)
+            mma_e4m3_ss_pv_k128(tmem + col_o(x, D), p_desc + ((x * C::kTileBytes) >> 4),
+                                v_desc + ((vslot * C::kTileBytes) >> 4), idesc_pv, first ? 0u : 1u);
+        else
+            mma_ts_k128(tmem + col_o(x, D), tmem + col_p_sep(x), v_desc + ((vslot * C::kTileBytes) >> 4), idesc_pv,
+                        first ? 0u : 1u);
         tc_commit(&bars[C::kBarPvDone + x]);
         return true;
     };
@@ -593,7 +604,7 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
         if (!mbar_wait(&bars[C::kBarQFull], tq & 1, abort_flag, to)) { ok = false; break; }
         ++tq;
         tc_fence_after();
-        if constexpr (kSepP<D> && !F8) {
+        if constexpr (kSepChain<D, F8>) {
             for (int j = 0; j <= u.nmax && ok; ++j) {
                 if (j < u.nmax) {
                     const uint32_t kslot = gk % C::kKStages;
@@ -636,12 +647,8 @@ __device__ __forceinline__ bool mma_role(const FwdParams &p, uint64_t *bars, vol
             if (j > 0 && j - 1 < u.n[0] && !pv(0, gp0, tl0, vslot, j == 1, j == u.n[0])) { ok = false; break; }
             if (have_k && j < u.n[0]) qk(0, kslot);
             if (j > 0 && j - 1 < u.n[1] && !pv(1, gp1, tl1, vslot, j == 1, j == u.n[1])) { ok = false; break; }
-            if (kEarlyVRelease<F8> && j > 0) {
-                tc_commit(&bars[C::kBarVEmpty + vslot]);
-                ++gv;
-            }
             if (have_k && j < u.n[1]) qk(1, kslot);
-            if (!kEarlyVRelease<F8> && j > 0) {
+            if (j > 0) {
                 tc_commit(&bars[C::kBarVEmpty + vslot]);
                 ++gv;
             }
@@ -808,14 +815,16 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_sm100_kernel(const __grid_
     if (warp < kSoftmaxWarps) {
         setmaxnreg_inc<kSoftmaxRegs>();
         uint8_t *stage = smem + C::kOffStage + warp * C::kStageBytes;
-        if (!softmax_role<D, O_BF16, F8>(p, bars, abort_flag, uq, tmem, warp >> 2, warp, lane, stage))
+        if (!softmax_role<D, O_BF16, F8>(p, bars, abort_flag, uq, tmem, warp >> 2, warp, lane, stage,
+                                         smem + C::kOffP))
             record_timeout(p);
     } else {
         setmaxnreg_dec<kControlRegs>();
     }
     if (warp == kMmaWarp) {
         if (lane == 0) {
-            if (!mma_role<D, F8>(p, bars, abort_flag, uq, tmem, smem_u32(sQ), smem_u32(sK), smem_u32(sV)))
+            if (!mma_role<D, F8>(p, bars, abort_flag, uq, tmem, smem_u32(sQ), smem_u32(sK), smem_u32(sV),
+                                 smem_u32(smem + C::kOffP)))
                 record_timeout(p);
             // drain: no MMA may still be running when TMEM is released
             tc_commit(&bars[C::kBarDrain]);

@@ -434,6 +434,26 @@ __device__ __forceinline__ void mma_e4m3_ts_k128(uint32_t d_tmem, uint32_t a_tme
 }
 #undef FA_F8TS_STEP
 
+// O (+)= P V over 128 keys of E4M3 with P in shared memory: P K-major (one
+// 128-byte swizzle row of 128 keys per query row, 32 bytes per step of K = 32),
+// V MN-major as in mma_e4m3_ts_k128 (4096 bytes = 256 in 16-byte units per step).
+#define FA_F8SSPV_STEP(DA, DB)                               \
+    "add.s64 da, %1, " #DA ";\n\t"                          \
+    "add.s64 db, %2, " #DB ";\n\t"                          \
+    "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %3, pt;\n\t"
+__device__ __forceinline__ void mma_e4m3_ss_pv_k128(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                    uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .b64 da, db;\n\t.reg .pred p, pt;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 pt, 1, 1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t"
+        FA_F8SSPV_STEP(2, 256) FA_F8SSPV_STEP(4, 512) FA_F8SSPV_STEP(6, 768)
+        "}" ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+#undef FA_F8SSPV_STEP
+
 // Four fp32 values rounded to E4M3 (nearest even, saturating) and packed into
 // one 32-bit word, a in the lowest byte.
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {

@@ -168,6 +168,22 @@ def algorithmic_bytes(w, k_len) -> float:
     return eb * n_elem + 2 * eb * kv_rows * w.d + 4.0 * n_elem + 4.0 * w.B * w.H * w.N
 
 
+def memory_footprint(w, workspace_bytes: int = 0) -> dict:
+    """Device memory of one forward call against that of the plain definition
+    (page "FlashAttention (ES)", sections "El problema de la atencion estandar"
+    and "Resultados empiricos"): the fused path holds Q, K, V, O and lse only
+    (plus a key-split workspace; the library allocates nothing), while the
+    definition also materialises the score matrix S = Q K^T of every head,
+    B*H*N*N_k fp32 values (counted once: the softmax can overwrite S in place)."""
+    eb = 1 if w.dtype == "e4m3" else 2
+    io = (eb * w.B * w.H * w.N * w.d + 2 * eb * w.B * w.kv_heads * w.keys * w.d
+          + 4 * w.B * w.H * w.N * w.d + 4 * w.B * w.H * w.N)
+    scores = 4 * w.B * w.H * w.N * w.keys
+    fused = io + workspace_bytes
+    return {"fused_bytes": fused, "definition_bytes": io + scores, "score_matrix_bytes": scores,
+            "ratio": (io + scores) / fused}
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle samples during the timed region."""
     FIELDS = ["pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
@@ -625,7 +641,7 @@ def measure_per_config(args, local, peaks, num_sms):
             "tflops_p90_time": flops / (st["p90"] * 1e-3) / 1e12,
             "frac": tf / peak, "frac_of_burst": tf / burst, "frac_of_sustained": tf / sustained,
             "algorithmic_bytes": algorithmic_bytes(w, k_len), "traffic": measured_traffic(wid),
-            "clocks": clocks,
+            "clocks": clocks, "memory": memory_footprint(w),
         }
         if clocks and clocks.get("sm_mhz"):
             cp = clock_peak_tflops(num_sms, clocks["sm_mhz"])
@@ -780,6 +796,7 @@ def run_ours(args, world, rank, local):
         "e2e": e2e,
         "gpu_launches": args.steps * (2 if splits > 1 else 1),
         "clocks": clocks,
+        "memory": memory_footprint(w, int(ws.numel()) if ws is not None else 0),
     }
     if per_config is not None:
         line["per_config"] = per_config

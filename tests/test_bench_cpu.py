@@ -179,3 +179,20 @@ def test_guard_regions_catch_writes_past_either_end():
     g2.buf[GUARD_BYTES - 1] = 1  # one byte before the start
     with pytest.raises(AssertionError, match="1 guard bytes changed before"):
         g2.check("head")
+
+
+def test_memory_footprint_against_the_definition():
+    """The memory restatement: the fused path holds Q, K, V, O, lse; the plain
+    definition adds one fp32 score matrix per head (B*H*N*N_k values)."""
+    w = workloads.WORKLOADS[4]  # B1 H32 N16384 d128 causal
+    m = bench.memory_footprint(w)
+    io = 3 * 2 * 32 * 16384 * 128 + 4 * 32 * 16384 * 128 + 4 * 32 * 16384
+    assert m["fused_bytes"] == io == bench.algorithmic_bytes(w, None)
+    assert m["score_matrix_bytes"] == 4 * 32 * 16384 * 16384
+    assert m["definition_bytes"] == io + 4 * 32 * 16384 * 16384
+    assert abs(m["ratio"] - (io + 4 * 32 * 16384 ** 2) / io) < 1e-9 and m["ratio"] > 50
+    # a key-split workspace counts on the fused side; E4M3 inputs take one byte
+    m2 = bench.memory_footprint(w, workspace_bytes=1 << 20)
+    assert m2["fused_bytes"] == io + (1 << 20)
+    w9 = workloads.WORKLOADS[9]
+    assert bench.memory_footprint(w9)["fused_bytes"] == 3 * 32 * 16384 * 128 + 4 * 32 * 16384 * 128 + 4 * 32 * 16384

@@ -31,8 +31,9 @@
  *
  * Ownership: the caller owns every buffer.  The library allocates, frees and
  * synchronises nothing (except fa_read_device_status and fa_fwd_host, which
- * say so), holds no state beyond a per-device cache of properties and the
- * driver's tensor-map entry point, and is safe to call from several threads.
+ * say so), holds no state beyond a per-device cache of properties (and the two
+ * copy streams of fa_fwd_host) and the driver's tensor-map entry point, and is
+ * safe to call from several threads.
  *
  * Errors: argument errors are returned synchronously and launch nothing.
  * Device-side errors (a pipeline wait that exceeded its time limit) are
@@ -204,8 +205,19 @@ typedef struct {
  * fa_fwd_host -- end-to-end call on HOST buffers: copies q, k, v (and k_len)
  * host -> device into the caller's device buffers, runs fa_fwd_ex, copies o
  * and lse device -> host, and synchronises `stream` before returning.
- * One cudaMemcpyAsync per buffer.  If dev.dev_status is set, a device-side
- * error found after the copies is returned as its fa_status.
+ * A call whose copies total 64 MB or more, and that gives every SM at least
+ * two work units per piece, is cut into up to 8 pieces: whole batch elements
+ * (B > 1) or whole groups of query heads sharing a key/value head (B = 1).
+ * Piece c's copies in run on a copy-in stream, its fa_fwd_ex on `stream` once
+ * they have landed, and its copies out on a copy-out stream once the kernel is
+ * done, so that copies in both directions and the kernels of different pieces
+ * overlap (the two streams are created once per device and kept).  The
+ * result equals the single call's bit for bit (each piece is a valid
+ * fa_fwd_ex problem with the caller's options; a call that cannot be cut that
+ * way runs whole).  Host buffers should be pinned for the copies to overlap.
+ * Work queued earlier on `stream` completes before the first copy.  If
+ * dev.dev_status is set, a device-side error found after the copies is
+ * returned as its fa_status.
  */
 FA_EXPORT fa_status fa_fwd_host(const fa_fwd_host_params *p, void *stream);
 

@@ -249,6 +249,35 @@ def test_host_entry_point():
     assert torch.equal(oh, o2) and torch.equal(lh, l2)
 
 
+@pytest.mark.parametrize("B,H,H_kv,N,d,causal,padded", [
+    (1, 32, 32, 8192, 128, True, False),   # pieces of whole heads
+    (1, 32, 8, 8192, 128, True, False),    # pieces of key/value-head groups
+    (16, 16, 16, 2048, 64, False, True),   # pieces of whole batch elements, key padding
+])
+def test_host_entry_point_in_pieces(B, H, H_kv, N, d, causal, padded):
+    """A large fa_fwd_host call is cut into pieces whose copies and kernels
+    overlap on three streams; the result equals the device entry point's bit
+    for bit."""
+    g = torch.Generator().manual_seed(70 + d + H_kv)
+    q = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H_kv, N, d, generator=g).to(torch.bfloat16)
+    k_len = torch.randint(N // 2, N + 1, (B,), generator=g, dtype=torch.int32) if padded else None
+    dev = torch.device("cuda:0")
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.full((B, H, N, d), float("nan")).pin_memory()
+    lh = torch.full((B, H, N), float("nan")).pin_memory()
+    qd, kd, vd = (torch.empty_like(t, device=dev) for t in (q, k, v))
+    od = torch.empty(B, H, N, d, device=dev)
+    ld = torch.empty(B, H, N, device=dev)
+    kw = {}
+    if padded:
+        kw = dict(k_len_h=k_len.pin_memory(), k_len_d=torch.empty(B, dtype=torch.int32, device=dev))
+    fb.fa_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, causal, 1 / math.sqrt(d), **kw)
+    o2, l2 = run_gpu(q, k, v, causal, 1 / math.sqrt(d), k_len=None if k_len is None else k_len.tolist())
+    assert torch.equal(oh, o2) and torch.equal(lh, l2)
+
+
 def test_no_device_memory_allocated():
     """The library allocates nothing: free device memory is unchanged across
     a launch (O(N) memory, no N x N buffer, no workspace)."""

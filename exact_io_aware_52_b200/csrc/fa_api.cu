@@ -460,12 +460,12 @@ fa_status fa_fwd_ex(const fa_fwd_params *p, void *stream) {
     kp.causal = p->causal;
     if (e4m3_in(p)) {
         // value scales: Q K^T by descale_q * descale_k (folded into the softmax
-        // scale), O by descale_v.  Weights are 2^(x - m_ref + 8) with x at most
-        // tau above m_ref, so they stay at or below 2^(8 + tau) = 430.5 for
-        // tau = 0.75, under E4M3's largest finite value 448 (no saturation).
+        // scale), O by descale_v.  Weights are 2^(x - m_ref + 7) with x at most
+        // tau above m_ref, so they stay at or below 2^(7 + tau) = 430.5 for
+        // tau = 1.75, under E4M3's largest finite value 448 (no saturation).
         kp.scale_log2 = (float)((double)p->scale * descale(p->descale_q) * descale(p->descale_k) *
                                 1.4426950408889634074);
-        kp.tau = (p->flags & FA_FLAG_EAGER_RESCALE) ? 0.f : 0.75f;
+        kp.tau = (p->flags & FA_FLAG_EAGER_RESCALE) ? 0.f : 1.75f;
         kp.out_scale = descale(p->descale_v);
     } else {
         kp.scale_log2 = (float)((double)p->scale * 1.4426950408889634074);

@@ -370,9 +370,9 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) 
 // ------------------------------------------------------------------ softmax
 // One warpgroup, query tile x; thread owns row (warp % 4) * 32 + lane.
 // E4M3 probabilities are taken relative to m_ref - kF8Shift (so that they lie
-// in (0, 2^(8 + tau)], tau <= 0.75: below E4M3's largest value 448, and
-// normal in E4M3 down to 2^-14 of the reference).
-constexpr float kF8Shift = 8.f;
+// in (0, 2^(7 + tau)], tau <= 1.75: below E4M3's largest value 448, and
+// normal in E4M3 down to 2^-13 of the reference).
+constexpr float kF8Shift = 7.f;
 
 template <int D, bool O_BF16, bool F8>
 __device__ __forceinline__ bool softmax_role(const FwdParams &p, uint64_t *bars, volatile int *abort_flag,

@@ -81,11 +81,11 @@ typedef enum {
 /* Flags for fa_fwd_params.flags. */
 enum {
     /* Rescale the running output whenever a row maximum grows, instead of
-     * only when it grows by more than a factor 2^8 (bf16 inputs) or 2^0.75
+     * only when it grows by more than a factor 2^8 (bf16 inputs) or 2^1.75
      * (E4M3 inputs, whose weights must stay below E4M3's largest value), the
      * defaults.  Both are exact up to rounding; the default skips most
      * rescales, this one keeps the largest softmax weight of each row at
-     * exactly 1 (E4M3: 2^8) before rounding. */
+     * exactly 1 (E4M3: 2^7) before rounding. */
     FA_FLAG_EAGER_RESCALE = 1
 };
 

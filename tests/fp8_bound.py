@@ -3,13 +3,13 @@
 With E4M3 inputs the kernel computes Q K^T exactly up to fp32 accumulation
 (a product of two E4M3 values has at most 8 significant bits), but rounds the
 probabilities to E4M3 before the product with V.  It takes them relative to
-a reference r minus 8 (log2 units) that trails the running row maximum by at
-most tau (0.75, or 0 with eager rescaling): each weight 2^(8 + x_j - r) <=
+a reference r minus 7 (log2 units) that trails the running row maximum by at
+most tau (1.75, or 0 with eager rescaling): each weight 2^(7 + x_j - r) <=
 2^8.75 < 448 is rounded either relatively (|dp| <= u p, u = 2^-4, three
 mantissa bits, for weights >= 2^-6, E4M3's smallest normal) or absolutely
 (|dp| <= 2^-10, half the subnormal spacing 2^-9, below it).  A weight taken
 while the reference was smaller is only larger at rounding time and is then
-scaled down exactly.  In units of the true row maximum m (p'_j = 2^(8 + x_j -
+scaled down exactly.  In units of the true row maximum m (p'_j = 2^(7 + x_j -
 m)) the final reference lies delta, 0 <= delta <= tau, below m: the
 absolutely rounded weights are a subset of those with p'_j < 2^-6, and their
 error over the sum is at most 2^-10 / (2^delta L') <= 2^-10 / L'.  O is
@@ -29,7 +29,7 @@ import numpy as np
 U_E4M3 = 2.0 ** -4
 SUB_E4M3 = 2.0 ** -6     # smallest normal
 HALF_SUB_SPACING = 2.0 ** -10
-SHIFT = 8.0
+SHIFT = 7.0
 
 
 def bound_rows(q, k, v, causal: bool, scale: float, k_len=None, rows=None):

@@ -1,7 +1,9 @@
 """The E4M3 error bound (tests/fp8_bound.py) holds for the rounding it
-describes: probabilities taken relative to the row maximum minus 8, rounded
-to E4M3 by torch, O divided by the unrounded sum.  Checked against the fp64
-oracle on random and peaked rows, where it must also not be vacuous."""
+describes: probabilities taken relative to a reference up to tau below the row
+maximum, minus the shift, rounded to E4M3 by torch, O divided by the
+unrounded sum.  Checked against the fp64 oracle on random and peaked rows,
+with the reference at the maximum and lagging it, where it must also not be
+vacuous."""
 import math
 
 import numpy as np
@@ -11,10 +13,18 @@ import oracle
 from tests import fp8_bound
 
 
-def _emulate(q, k, v, scale):
-    """O of the rounding model: weights 2^(8 + x - max) rounded to E4M3."""
+TAU = 1.75  # the kernel's rescale threshold for E4M3 inputs (log2 units)
+
+
+def _emulate(q, k, v, scale, lag=None):
+    """O of the rounding model: weights 2^(SHIFT + x - r) rounded to E4M3, with
+    the reference r = max - lag (lag per row in [0, TAU]; 0 when None)."""
     x = torch.einsum("bhid,bhjd->bhij", q, k) * scale / math.log(2.0)
-    pp = torch.exp2(8.0 + x - x.amax(-1, keepdim=True))
+    r = x.amax(-1, keepdim=True)
+    if lag is not None:
+        r = r - lag
+    pp = torch.exp2(fp8_bound.SHIFT + x - r)
+    assert pp.max().item() <= 2.0 ** (fp8_bound.SHIFT + TAU) < 448.0
     pr = pp.float().to(torch.float8_e4m3fn).double()
     return torch.einsum("bhij,bhjd->bhid", pr, v) / pp.sum(-1, keepdim=True)
 
@@ -28,8 +38,10 @@ def test_bound_holds_for_the_rounding_model():
         scale = float(np.float32(1 / math.sqrt(128)))
         o_ref, _ = oracle.attention_f64(q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16), False,
                                         scale)
-        o_emul = _emulate(q.double(), k.double(), v.double(), scale).numpy().reshape(o_ref.shape)
         bound = fp8_bound.bound_rows(q.double().numpy(), k.double().numpy(), v.double().numpy(), False, scale)
-        err = np.abs(o_emul - o_ref)
-        assert np.all(err <= bound)
-        assert err.max() > 0.05 * bound.max()  # the bound is not vacuously loose here
+        lag = torch.rand(1, 2, 64, 1, generator=g, dtype=torch.float64) * TAU
+        for lg in (None, lag):
+            o_emul = _emulate(q.double(), k.double(), v.double(), scale, lg).numpy().reshape(o_ref.shape)
+            err = np.abs(o_emul - o_ref)
+            assert np.all(err <= bound)
+            assert err.max() > 0.05 * bound.max()  # the bound is not vacuously loose here

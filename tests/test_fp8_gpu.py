@@ -106,18 +106,18 @@ def test_large_logits(std, flags):
 
 @pytest.mark.parametrize("flags", [0, fb.FA_FLAG_EAGER_RESCALE])
 def test_slowly_growing_maximum(flags):
-    """Scores that grow along the keys by about 0.4 (head 0) and 1.0 (head 1)
-    natural units per key tile: the row maximum moves on most tiles, often by
-    less than the rescale threshold (weights then reach up to 2^8.75 before
-    rounding) and often by more."""
+    """Scores that grow along the keys by about 0.8 (head 0) and 1.6 (head 1)
+    natural units per key tile (1.2 and 2.3 binary orders): the row maximum
+    moves on most tiles, often by less than the rescale threshold 1.75
+    (weights then reach up to 2^8.75 before rounding) and often by more."""
     B, H, N = 1, 2, 1024
     g = torch.Generator().manual_seed(3010 + flags)
     q = torch.zeros(B, H, N, D)
     k = torch.zeros(B, H, N, D)
     q[..., 0] = 1.0
     q[..., 1] = 0.5
-    k[0, 0, :, 0] = torch.linspace(0.0, 0.4 * N / 128, N)
-    k[0, 1, :, 0] = torch.linspace(0.0, 1.0 * N / 128, N)
+    k[0, 0, :, 0] = torch.linspace(0.0, 0.8 * N / 128, N)
+    k[0, 1, :, 0] = torch.linspace(0.0, 1.6 * N / 128, N)
     k[..., 1] = torch.randn(B, H, N, generator=g)
     v = torch.randn(B, H, N, D, generator=g)
     q, k, v = (t.to(torch.float8_e4m3fn) for t in (q, k, v))
